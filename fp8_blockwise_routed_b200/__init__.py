@@ -1,0 +1,195 @@
+"""Python binding of libfp8moe.so: the B200 routed-MoE FP8 blockwise (W8A8)
+prefill path.
+
+Functions named after the C ABI (include/fp8moe.h) marshal torch tensors
+into pointers and the current CUDA stream; every step of the path runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams only.
+There is no fallback: if the library is missing or the device is not an
+sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8moe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "fp8moe.h")
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_ALIGNMENT",
+          4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_DEVICE_STATUS"}
+DEV_BAD_EXPERT_ID, DEV_BAD_PAIR, DEV_BAD_OFFSETS, DEV_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions the public header declares."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m fp8_blockwise_routed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [i32]
+        L.moe_abi_version.restype = i32
+        L.moe_route_workspace_bytes.restype = sz
+        L.moe_route_workspace_bytes.argtypes = [i64, i32, i32]
+        L.moe_route.restype = i32
+        L.moe_route.argtypes = [P, i64, i32, i32, P, P, P, P, P, sz, P]
+        L.moe_quant_act.restype = i32
+        L.moe_quant_act.argtypes = [P, i64, i32, P, P, P]
+        L.moe_ffn_workspace_bytes.restype = sz
+        L.moe_ffn_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+        L.moe_grouped_ffn.restype = i32
+        L.moe_grouped_ffn.argtypes = [P, P, i64, i32, P, P, i32, P, P, i32, i32,
+                                      P, P, P, P, P, P, P, P, sz, P]
+        L.moe_combine_workspace_bytes.restype = sz
+        L.moe_combine_workspace_bytes.argtypes = []
+        L.moe_combine.restype = i32
+        L.moe_combine.argtypes = [P, P, i64, i32, i32, i32, ctypes.c_float, P, P, P, sz, P]
+        L.moe_get_device_status.restype = i32
+        L.moe_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+        L.moe_debug_encode.restype = i32
+        L.moe_debug_encode.argtypes = [P, i64, P, P]
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise MoeError(code, what)
+
+
+# ------------------------------------------------------------------ sizes
+
+def moe_route_workspace_bytes(T: int, E: int, top_k: int) -> int:
+    return int(lib().moe_route_workspace_bytes(T, E, top_k))
+
+
+def moe_ffn_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> int:
+    return int(lib().moe_ffn_workspace_bytes(T, H, I, E, top_k))
+
+
+def moe_combine_workspace_bytes() -> int:
+    return int(lib().moe_combine_workspace_bytes())
+
+
+# ------------------------------------------------------------------ calls
+
+def moe_route(logits, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, stream=None):
+    T, E = logits.shape
+    _check(lib().moe_route(_p(logits), T, E, top_k, _p(topk_ids), _p(topk_w), _p(expert_offsets),
+                           _p(sorted_pairs), _p(ws), ws.numel() * ws.element_size(), _s(stream)), "moe_route")
+
+
+def moe_quant_act(x, codes, scales, stream=None):
+    T, H = x.shape
+    _check(lib().moe_quant_act(_p(x), T, H, _p(codes), _p(scales), _s(stream)), "moe_quant_act")
+
+
+def moe_grouped_ffn(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs,
+                    w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None):
+    T, H = codes.shape
+    E, I, _ = w_gate.shape
+    top_k = topk_ids.shape[1]
+    _check(lib().moe_grouped_ffn(_p(codes), _p(act_scales), T, H, _p(topk_ids), _p(topk_w), top_k,
+                                 _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate),
+                                 _p(w_up), _p(s_up), _p(w_down), _p(s_down), _p(y), _p(ws),
+                                 ws.numel() * ws.element_size(), _s(stream)), "moe_grouped_ffn")
+
+
+def moe_combine(y, topk_ids, num_experts, routed_scaling, out_f32, out_bf16, ws, stream=None):
+    T, top_k = topk_ids.shape
+    H = out_f32.shape[1]
+    _check(lib().moe_combine(_p(y), _p(topk_ids), T, H, top_k, num_experts, float(routed_scaling),
+                             _p(out_f32), _p(out_bf16), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "moe_combine")
+
+
+def moe_get_device_status(ws) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().moe_get_device_status(_p(ws), ctypes.byref(v)), "moe_get_device_status")
+    return int(v.value)
+
+
+def moe_debug_encode(inp, out, stream=None):
+    _check(lib().moe_debug_encode(_p(inp), inp.numel(), _p(out), _s(stream)), "moe_debug_encode")
+
+
+# ------------------------------------------------------------------ layer
+
+class RoutedMoE:
+    """One routed-expert layer: resident FP8 weights and their block scales,
+    plus output and workspace buffers sized for up to `max_tokens` rows.
+    ``forward`` enqueues moe_quant_act, moe_route, moe_grouped_ffn and
+    moe_combine on the current stream and returns the FP32 output rows."""
+
+    def __init__(self, w_gate, s_gate, w_up, s_up, w_down, s_down, top_k: int, routed_scaling: float,
+                 max_tokens: int):
+        self.w = (w_gate, s_gate, w_up, s_up, w_down, s_down)
+        self.E, self.I, self.H = w_gate.shape
+        self.k = int(top_k)
+        self.rs = float(routed_scaling)
+        self.max_tokens = int(max_tokens)
+        dev = w_gate.device
+        T, H, E, k = self.max_tokens, self.H, self.E, self.k
+        u8, i32, f32 = torch.uint8, torch.int32, torch.float32
+        self.codes = torch.empty((T, H), dtype=u8, device=dev)
+        self.scales = torch.empty((T, H // 128), dtype=f32, device=dev)
+        self.ids = torch.empty((T, k), dtype=i32, device=dev)
+        self.tw = torch.empty((T, k), dtype=f32, device=dev)
+        self.offsets = torch.empty((E + 1,), dtype=i32, device=dev)
+        self.sorted = torch.empty((T * k,), dtype=i32, device=dev)
+        self.y = torch.empty((T, k, H), dtype=f32, device=dev)
+        self.out = torch.empty((T, H), dtype=f32, device=dev)
+        self.ws_route = torch.empty((moe_route_workspace_bytes(T, E, k),), dtype=u8, device=dev)
+        self.ws_ffn = torch.empty((moe_ffn_workspace_bytes(T, H, self.I, E, k),), dtype=u8, device=dev)
+        self.ws_comb = torch.empty((moe_combine_workspace_bytes(),), dtype=u8, device=dev)
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, out_bf16: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        assert T <= self.max_tokens and x.shape[1] == self.H and logits.shape == (T, self.E)
+        codes, scales = self.codes[:T], self.scales[:T]
+        ids, tw, srt = self.ids[:T], self.tw[:T], self.sorted[: T * self.k]
+        y, out = self.y[:T], self.out[:T]
+        moe_quant_act(x, codes, scales, stream)
+        moe_route(logits, self.k, ids, tw, self.offsets, srt, self.ws_route, stream)
+        moe_grouped_ffn(codes, scales, ids, tw, self.offsets, srt, *self.w, y, self.ws_ffn, stream)
+        moe_combine(y, ids, self.E, self.rs, out, out_bf16, self.ws_comb, stream)
+        return out
+
+    def device_status(self) -> int:
+        return (moe_get_device_status(self.ws_route) | moe_get_device_status(self.ws_ffn)
+                | moe_get_device_status(self.ws_comb))

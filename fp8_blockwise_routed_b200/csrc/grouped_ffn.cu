@@ -1,0 +1,616 @@
+// grouped_ffn.cu -- the expert FFN of the routed-MoE W8A8 prefill path on
+// sm_100a tensor cores (tcgen05 + TMEM, operands fed by TMA).
+//
+// Pages: blockwise FP8 MoE with 128x128 weight scales and zero-padding of a
+// non-128-divisible intermediate ("Integration for GLM-4.6-FP8 and
+// performance tune on H20", gap table row 6), single-wave grid sizing (row
+// 3); unclamped SiLU, W8A8 ("Full GLM-5.3 streamed FP8 GPU prefill ...",
+// "Design"); whole-K accumulation without split-K, fixed member order, routed
+// FP32 rows written in place, one call per prompt pass ("GLM-5.3-Flash EXL3
+// on CUDA: a whole prompt pass routes its experts in one call").
+//
+// Launch sequence of one moe_grouped_ffn call (stream-ordered, no host sync):
+//   gather   : A rows in expert order: a_sorted[r] = codes[token(r)],
+//              sa_sorted[r] = act_scales[token(r)]             (HBM/L2-bound)
+//   gate/up  : persistent grouped GEMM, tile = 128 pair rows x (128 gate +
+//              128 up) columns, one MMA of N=256 per 32-wide K step; epilogue
+//              h = SiLU(g)*u, requantised per 128-group -> h codes/scales
+//   down     : same kernel, tile = 128 rows x 256 output columns over the
+//              intermediate; epilogue y[pair] = w_pair * o
+//
+// Block scales (FP32, not powers of two) have no tensor-core path, so every
+// 128-deep K block is its own MMA chain into a fresh TMEM accumulator
+// ("partial"), and the epilogue warps fold it into FP32 registers with
+//   acc += (sa[row,kb] * sw[nblock,kb]) * partial.
+// Two partial buffers of 256 TMEM columns alternate, so the MMA of block kb+1
+// overlaps the promotion of block kb.
+//
+// Warp roles (320 threads, one CTA per SM, grid = #SMs, static round-robin
+// over work items ordered expert-major, then n-tile, then m-tile so that the
+// m-tiles sharing a weight panel run at the same time and share it in L2):
+//   warp 0      TMA producer (one lane): A tile 128x128 B, B tile 2x128x128 B
+//               per stage, 4 stages, mbarrier complete_tx
+//   warp 1      TMEM allocator and MMA issuer (one lane)
+//   warps 2..9  promotion + epilogue; warp w reads TMEM lanes 32*(w%4) (its
+//               rows); warps 2..5 own columns [0,64) of each 128-half, warps
+//               6..9 columns [64,128)
+// Every wait is bounded (2 s of global time); on expiry the CTA raises an
+// abort flag, records MOE_DEV_WAIT_TIMEOUT, drains and frees TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cfloat>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fp8moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BK = 128;
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK;           // 16 KiB
+constexpr int B_HALF = 128 * BK;          // 16 KiB
+constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr int MAX_E = 1024;
+
+// shared memory map (after the 1024-aligned stage ring)
+constexpr int OFF_BARS = STAGES * STAGE_BYTES;
+constexpr int N_BARS = 2 * STAGES + 4 + 4;  // full, empty, tfull[2], tempty[2], xbar[4]
+constexpr int OFF_MISC = OFF_BARS + N_BARS * 8;
+constexpr int OFF_AMAX = OFF_MISC + 16;                  // [2 parity][2 half][128 rows] floats
+constexpr int OFF_SEG = OFF_AMAX + 2 * 2 * 128 * 4;      // [MAX_E+1] ints
+constexpr int OFF_IPRE = OFF_SEG + (MAX_E + 1) * 4;      // [MAX_E+1] ints
+constexpr int SMEM_USED = OFF_IPRE + (MAX_E + 1) * 4;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;              // slack for 1024-alignment
+
+struct GemmParams {
+    int E;
+    int num_kb;            // K blocks of 128
+    int n_tiles;           // output tiles per expert along N
+    int64_t P;             // rows of the pair buffers (T * top_k)
+    const int32_t* offsets;
+    const float* a_scales; // [P, num_kb] in expert order
+    const float* b_s0;     // gate/up: s_gate; down: s_down
+    const float* b_s1;     // gate/up: s_up;   down: s_down
+    int b_nblocks;         // scale n-blocks per expert (ceil(I/128) or H/128)
+    // gate/up epilogue
+    uint8_t* h_codes;      // [P, Ip]
+    float* h_scales;       // [P, GI]
+    int Ip;
+    int GI;
+    // down epilogue
+    const int32_t* sorted_pairs;
+    const float* topk_w;
+    float* y;              // [P, H]
+    int H;
+    int* status;
+};
+
+__device__ __forceinline__ int find_expert(const int* ipre, int E, int item)
+{
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ipre[mid] <= item) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+struct Item {
+    int e, nt, mt;
+};
+
+__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item)
+{
+    Item it;
+    it.e = find_expert(ipre, E, item);
+    const int local = item - ipre[it.e];
+    const int mts = (seg[it.e + 1] - seg[it.e] + BM - 1) / BM;
+    it.nt = local / mts;
+    it.mt = local - it.nt * mts;
+    return it;
+}
+
+// ---------------------------------------------------------------- roles
+
+template <int MODE>
+__device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB0, const CUtensorMap* tmB1,
+                              const GemmParams& p, const int* seg, const int* ipre, int total_items,
+                              uint32_t sbase, uint32_t bars, volatile int* abort)
+{
+    const uint32_t full0 = bars, empty0 = bars + STAGES * 8;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        const Item w = decode_item(seg, ipre, p.E, item);
+        const int row0 = seg[w.e] + w.mt * BM;
+        const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
+        const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort, WAIT_NS)) {
+                ok = false;
+                break;
+            }
+            const uint32_t fb = full0 + 8 * s;
+            mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            const uint32_t a_dst = sbase + s * STAGE_BYTES;
+            tma_load_2d(a_dst, tmA, kb * BK, row0, fb);
+            tma_load_3d(a_dst + A_TILE, tmB0, kb * BK, n0, w.e, fb);
+            tma_load_3d(a_dst + A_TILE + B_HALF, tmB1, kb * BK, n1, w.e, fb);
+        }
+    }
+    if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        const int first = it - STAGES > 0 ? it - STAGES : 0;
+        for (int j = first; j < it; ++j) {
+            volatile int no_abort = 0;
+            mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1, &no_abort, WAIT_NS / 4);
+        }
+    }
+}
+
+__device__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         volatile int* abort)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t full0 = bars, empty0 = bars + STAGES * 8;
+    const uint32_t tfull0 = bars + 2 * STAGES * 8, tempty0 = tfull0 + 16;
+    constexpr uint32_t idesc = idesc_e4m3_f32(128, 256);
+    int it = 0;
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            const int b = it & 1;
+            const uint32_t bph = (it >> 1) & 1;
+            // every lane waits; the outcome is made warp-uniform so that no
+            // lane is left behind in a warp-synchronous instruction
+            bool ok = mbar_wait_bounded(tempty0 + 8 * b, bph ^ 1, abort, WAIT_NS);
+            ok = ok && mbar_wait_bounded(full0 + 8 * s, ph, abort, WAIT_NS);
+            if (!__all_sync(0xFFFFFFFFu, ok)) goto drain;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t a_addr = sbase + s * STAGE_BYTES;
+                const uint32_t b_addr = a_addr + A_TILE;
+                const uint32_t d = tmem + b * 256;
+#pragma unroll
+                for (int kk = 0; kk < BK / 32; ++kk)
+                    mma_f8(d, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(empty0 + 8 * s);
+                mma_commit(tfull0 + 8 * b);
+            }
+            __syncwarp();
+        }
+    }
+    return;
+drain:
+    // wait for the MMAs already issued before TMEM is released
+    if (it > 0) {
+        volatile int no_abort = 0;
+        const int last = it - 1;
+        mbar_wait_bounded(tfull0 + 8 * (last & 1), (last >> 1) & 1, &no_abort, WAIT_NS / 4);
+    }
+}
+
+template <int MODE>
+__device__ void epilogue_role(const GemmParams& p, const int* seg, const int* ipre, int total_items, uint32_t bars,
+                              uint32_t tmem, float* amax_x, volatile int* abort)
+{
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;        // column half-slice of each 128-wide half
+    const int trow = q * 32 + lane;          // row within the tile
+    const uint32_t tfull0 = bars + 2 * STAGES * 8, tempty0 = tfull0 + 16, xbar0 = tempty0 + 16;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    int it = 0;
+    int nitem = 0;
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++nitem) {
+        const Item w = decode_item(seg, ipre, p.E, item);
+        const int r = seg[w.e] + w.mt * BM + trow;
+        const bool valid = r < seg[w.e + 1];
+        const int64_t ra = r < p.P ? r : p.P - 1;
+        const float* sa_row = p.a_scales + ra * p.num_kb;
+        int nb0, nb1;
+        if (MODE == 0) {
+            nb0 = nb1 = w.nt;
+        } else {
+            nb0 = 2 * w.nt;
+            nb1 = 2 * w.nt + 1;
+        }
+        const float* s0 = p.b_s0 + (static_cast<int64_t>(w.e) * p.b_nblocks + nb0) * p.num_kb;
+        const float* s1 = p.b_s1 + (static_cast<int64_t>(w.e) * p.b_nblocks + (nb1 < p.b_nblocks ? nb1 : nb0)) * p.num_kb;
+        const bool has1 = nb1 < p.b_nblocks;
+
+        float acc0[64], acc1[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            acc0[i] = 0.f;
+            acc1[i] = 0.f;
+        }
+        float sa_next = __ldg(sa_row);
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            const int b = it & 1;
+            const uint32_t bph = (it >> 1) & 1;
+            const float sa = sa_next;
+            if (kb + 1 < p.num_kb) sa_next = __ldg(sa_row + kb + 1);
+            const float c0 = sa * __ldg(s0 + kb);
+            const float c1 = has1 ? sa * __ldg(s1 + kb) : 0.f;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, bph, abort, WAIT_NS))) return;
+            tc_fence_after();
+            const uint32_t col = lane_base + b * 256 + half * 64;
+            float v[32];
+            tmem_ld32(col, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc0[i] = fmaf(c0, v[i], acc0[i]);
+            tmem_ld32(col + 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc0[32 + i] = fmaf(c0, v[i], acc0[32 + i]);
+            tmem_ld32(col + 128, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc1[i] = fmaf(c1, v[i], acc1[i]);
+            tmem_ld32(col + 160, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(c1, v[i], acc1[32 + i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty0 + 8 * b);
+        }
+
+        if (MODE == 0) {
+            // h = SiLU(g) * u (unclamped), then the 1x128 group quantiser over
+            // this row's 128 intermediate columns [nt*128, nt*128+128), half of
+            // which this thread holds; the other half comes through shared
+            // memory from the partner warp of the same lane quarter.
+            float amax = 0.f;
+            int bad = 0;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float g = acc0[i];
+                const float h = __fdiv_rn(g, 1.0f + expf(-g)) * acc1[i];
+                acc0[i] = h;
+                if (isfinite(h)) amax = fmaxf(amax, fabsf(h));
+                else bad = 1;
+            }
+            const int par = nitem & 1;
+            amax_x[(par * 2 + half) * 128 + trow] = bad ? INFINITY : amax;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xbar0 + 8 * q);
+            if (!__all_sync(0xFFFFFFFFu,
+                            mbar_wait_bounded(xbar0 + 8 * q, static_cast<uint32_t>(nitem & 1), abort, WAIT_NS)))
+                return;
+            const float other = amax_x[(par * 2 + (half ^ 1)) * 128 + trow];
+            const bool nonfinite = bad || isinf(other);
+            float s = __fdiv_rn(fmaxf(amax, other), 448.0f);
+            if (s == 0.f) s = 1.f;
+            if (valid) {
+                uint8_t* dst = p.h_codes + static_cast<int64_t>(r) * p.Ip + w.nt * 128 + half * 64;
+                if (nonfinite) {
+                    s = __int_as_float(0x7FC00000);
+                    const uint4 nanq = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) reinterpret_cast<uint4*>(dst)[c] = nanq;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t wv[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int i = c * 16 + j * 4;
+                            const uint32_t lo = e4m3x2(__fdiv_rn(acc0[i], s), __fdiv_rn(acc0[i + 1], s));
+                            const uint32_t hi = e4m3x2(__fdiv_rn(acc0[i + 2], s), __fdiv_rn(acc0[i + 3], s));
+                            wv[j] = lo | (hi << 16);
+                        }
+                        reinterpret_cast<uint4*>(dst)[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    }
+                }
+                if (half == 0) p.h_scales[static_cast<int64_t>(r) * p.GI + w.nt] = s;
+            }
+        } else {
+            if (valid) {
+                const int pair = __ldg(p.sorted_pairs + r);
+                if (pair < 0 || pair >= p.P) {
+                    atomicOr(p.status, kDevBadPair);
+                } else {
+                    const float wt = __ldg(p.topk_w + pair);
+                    float* dst = p.y + static_cast<int64_t>(pair) * p.H;
+                    const int c0 = w.nt * 256 + half * 64;
+                    const int c1 = c0 + 128;
+                    if (c0 < p.H) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            reinterpret_cast<float4*>(dst + c0)[c] =
+                                make_float4(wt * acc0[4 * c], wt * acc0[4 * c + 1], wt * acc0[4 * c + 2],
+                                            wt * acc0[4 * c + 3]);
+                    }
+                    if (c1 < p.H) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            reinterpret_cast<float4*>(dst + c1)[c] =
+                                make_float4(wt * acc1[4 * c], wt * acc1[4 * c + 1], wt * acc1[4 * c + 2],
+                                            wt * acc1[4 * c + 3]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __maxnreg__(200)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bars = sbase + OFF_BARS;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+    int* bad = reinterpret_cast<int*>(smem + OFF_MISC + 8);
+    float* amax_x = reinterpret_cast<float*>(smem + OFF_AMAX);
+    int* seg = reinterpret_cast<int*>(smem + OFF_SEG);
+    int* ipre = reinterpret_cast<int*>(smem + OFF_IPRE);
+    const int warp = threadIdx.x >> 5;
+    const int E = p.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bars + 8 * s, 1);                 // full: producer arrive + tx
+            mbar_init(bars + 8 * (STAGES + s), 1);      // empty: MMA commit
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars + 8 * (2 * STAGES + b), 1);              // tfull: MMA commit
+            mbar_init(bars + 8 * (2 * STAGES + 2 + b), EPI_WARPS);  // tempty: epilogue warps
+        }
+        for (int q = 0; q < 4; ++q) mbar_init(bars + 8 * (2 * STAGES + 4 + q), 2);  // amax exchange
+        *abort = 0;
+        *bad = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && threadIdx.x == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB0);
+        prefetch_tmap(&tmB1);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) seg[i] = __ldg(p.offsets + i);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int okv = (seg[0] == 0);
+        int acc = 0;
+        ipre[0] = 0;
+        for (int e = 0; e < E; ++e) {
+            const int c = seg[e + 1] - seg[e];
+            if (c < 0 || seg[e + 1] > p.P) okv = 0;
+            const int mts = c > 0 ? (c + BM - 1) / BM : 0;
+            acc += mts * p.n_tiles;
+            ipre[e + 1] = acc;
+        }
+        if (!okv) {
+            *bad = 1;
+            if (blockIdx.x == 0) atomicOr(p.status, kDevBadOffsets);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total_items = *bad ? 0 : ipre[E];
+
+    if (warp == 0) {
+        if ((threadIdx.x & 31) == 0)
+            producer_role<MODE>(&tmA, &tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
+    } else if (warp == 1) {
+        mma_role(p, total_items, sbase, bars, tmem, abort);
+    } else {
+        epilogue_role<MODE>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && *abort) atomicOr(p.status, kDevWaitTimeout);
+}
+
+// Gather: one warp per sorted row r < P_valid copies the token's code row
+// and scale row into expert order.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restrict__ codes,
+                                                          const float* __restrict__ act_scales, int H, int k,
+                                                          const int32_t* __restrict__ sorted_pairs,
+                                                          const int32_t* __restrict__ offsets, int E, int64_t P,
+                                                          uint8_t* __restrict__ a_sorted,
+                                                          float* __restrict__ sa_sorted, int* __restrict__ status)
+{
+    const int lane = threadIdx.x & 31;
+    int64_t nvalid = offsets[E];
+    if (nvalid > P || nvalid < 0) nvalid = 0;  // the GEMM reports inconsistent offsets
+    const int GH = H / 128;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r = warp; r < nvalid; r += nwarps) {
+        const int pair = __ldg(sorted_pairs + r);
+        if (pair < 0 || pair >= P) {
+            if (lane == 0) atomicOr(status, kDevBadPair);
+            continue;
+        }
+        const int64_t t = pair / k;
+        const uint4* src = reinterpret_cast<const uint4*>(codes + t * H);
+        uint4* dst = reinterpret_cast<uint4*>(a_sorted + r * H);
+        for (int c = lane; c < H / 16; c += 32) dst[c] = __ldg(src + c);
+        for (int c = lane; c < GH; c += 32) sa_sorted[r * GH + c] = __ldg(act_scales + t * GH + c);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Row-major uint8 tensor of `rank` dims (innermost first), tile box of
+// 128 bytes x box_rows (x 1), 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+               uint32_t box_rows)
+{
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t gdim[3], gstr[2];
+    cuuint32_t box[3], estr[3];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        estr[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+    box[0] = 128;
+    box[1] = box_rows;
+    if (rank == 3) box[2] = 1;
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), gdim, gstr, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
+                     int grid, cudaStream_t s)
+{
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (err != cudaSuccess) return err;
+        attr_done[dev] = true;
+    }
+    grouped_gemm_kernel<MODE><<<grid, THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
+                            size_t* off_sh)
+{
+    const int64_t P = T * k > 0 ? T * k : 1;
+    const int GI = (I + 127) / 128;
+    const int64_t Ip = static_cast<int64_t>(GI) * 128;
+    size_t o = 256;  // status word
+    *off_a = o;
+    o = align_up(o + static_cast<size_t>(P) * H, 256);
+    *off_sa = o;
+    o = align_up(o + static_cast<size_t>(P) * (H / 128) * 4, 256);
+    *off_h = o;
+    o = align_up(o + static_cast<size_t>(P) * Ip, 256);
+    *off_sh = o;
+    o = align_up(o + static_cast<size_t>(P) * GI * 4, 256);
+    return o;
+}
+
+cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
+{
+    const int64_t P = a.T * a.k;
+    if (P == 0) return cudaSuccess;
+    DeviceInfo di;
+    if (!device_info(&di)) return cudaErrorUnknown;
+    if (di.max_smem_optin < static_cast<size_t>(SMEM_BYTES)) return cudaErrorNotSupported;
+    const int H = a.H, I = a.I, E = a.E;
+    const int GH = H / 128, GI = (I + 127) / 128, Ip = GI * 128;
+
+    // 1. gather the A operand rows (and their scales) into expert order
+    {
+        const int64_t want = ceil_div64(P, 8);
+        const int64_t cap = static_cast<int64_t>(di.sm_count) * 16;
+        gather_rows_kernel<<<static_cast<int>(want < cap ? want : cap), 256, 0, s>>>(
+            a.codes, a.act_scales, H, a.k, a.sorted_pairs, a.expert_offsets, E, P, a.a_sorted, a.sa_sorted,
+            a.status);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+
+    // 2. tensor maps
+    CUtensorMap tmA1, tmG, tmU, tmA2, tmD;
+    {
+        const uint64_t dA[2] = {static_cast<uint64_t>(H), static_cast<uint64_t>(P)};
+        const uint64_t sA[1] = {static_cast<uint64_t>(H)};
+        const uint64_t dW[3] = {static_cast<uint64_t>(H), static_cast<uint64_t>(I), static_cast<uint64_t>(E)};
+        const uint64_t sW[2] = {static_cast<uint64_t>(H), static_cast<uint64_t>(I) * H};
+        const uint64_t dH[2] = {static_cast<uint64_t>(Ip), static_cast<uint64_t>(P)};
+        const uint64_t sH[1] = {static_cast<uint64_t>(Ip)};
+        const uint64_t dD[3] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H), static_cast<uint64_t>(E)};
+        const uint64_t sD[2] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H) * I};
+        if (!make_tmap(&tmA1, a.a_sorted, 2, dA, sA, 128) || !make_tmap(&tmG, a.w_gate, 3, dW, sW, 128) ||
+            !make_tmap(&tmU, a.w_up, 3, dW, sW, 128) || !make_tmap(&tmA2, a.h_codes, 2, dH, sH, 128) ||
+            !make_tmap(&tmD, a.w_down, 3, dD, sD, 128))
+            return cudaErrorNotSupported;
+    }
+    const int grid = di.sm_count;
+
+    // 3. gate/up GEMM with the SiLU*up + requantisation epilogue
+    GemmParams g{};
+    g.E = E;
+    g.num_kb = GH;
+    g.n_tiles = GI;
+    g.P = P;
+    g.offsets = a.expert_offsets;
+    g.a_scales = a.sa_sorted;
+    g.b_s0 = a.s_gate;
+    g.b_s1 = a.s_up;
+    g.b_nblocks = GI;
+    g.h_codes = a.h_codes;
+    g.h_scales = a.h_scales;
+    g.Ip = Ip;
+    g.GI = GI;
+    g.sorted_pairs = a.sorted_pairs;
+    g.topk_w = a.topk_w;
+    g.y = a.y;
+    g.H = H;
+    g.status = a.status;
+    cudaError_t err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
+    if (err != cudaSuccess) return err;
+
+    // 4. down GEMM with the routing-weighted row epilogue
+    GemmParams d = g;
+    d.num_kb = GI;
+    d.n_tiles = (H + 255) / 256;
+    d.a_scales = a.h_scales;
+    d.b_s0 = a.s_down;
+    d.b_s1 = a.s_down;
+    d.b_nblocks = GH;
+    return run_gemm<1>(tmA2, tmD, tmD, d, grid, s);
+}
+
+}  // namespace fp8moe

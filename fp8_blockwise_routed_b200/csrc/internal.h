@@ -1,0 +1,73 @@
+// internal.h -- launchers shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8moe {
+
+// Status bits written by kernels (same values as the MOE_DEV_* macros of the
+// public header).
+constexpr int kDevBadExpertId = 0x1;
+constexpr int kDevBadPair = 0x2;
+constexpr int kDevBadOffsets = 0x4;
+constexpr int kDevWaitTimeout = 0x8;
+
+// Route kernels: tokens per routing block (8 warps x 16 tokens).
+constexpr int kRouteTokensPerBlock = 128;
+
+inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct DeviceInfo {
+    int sm_count;
+    int major, minor;
+    size_t max_smem_optin;
+};
+// Cached per device; returns false if the current device cannot be queried.
+bool device_info(DeviceInfo* out);
+
+cudaError_t launch_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* scales, cudaStream_t s);
+cudaError_t launch_encode(const float* in, int64_t n, uint8_t* out, cudaStream_t s);
+
+cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w,
+                         int32_t* offsets, int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank,
+                         cudaStream_t s);
+
+cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
+                           float* out, uint16_t* out_bf16, int* status, cudaStream_t s);
+
+struct FfnArgs {
+    const uint8_t* codes;
+    const float* act_scales;
+    int64_t T;
+    int H;
+    const int32_t* topk_ids;
+    const float* topk_w;
+    int k;
+    const int32_t* expert_offsets;
+    const int32_t* sorted_pairs;
+    int E;
+    int I;
+    const uint8_t* w_gate;
+    const float* s_gate;
+    const uint8_t* w_up;
+    const float* s_up;
+    const uint8_t* w_down;
+    const float* s_down;
+    float* y;
+    // workspace pieces
+    int* status;
+    uint8_t* a_sorted;   // [P, H]
+    float* sa_sorted;    // [P, H/128]
+    uint8_t* h_codes;    // [P, Ip]
+    float* h_scales;     // [P, ceil(I/128)]
+};
+size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
+                            size_t* off_sh);
+// Returns cudaSuccess, or an error (including cudaErrorNotSupported when the
+// tensor-map encoder cannot be obtained).
+cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s);
+
+}  // namespace fp8moe

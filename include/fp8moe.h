@@ -1,0 +1,241 @@
+/*
+ * fp8moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts FP8
+ * blockwise (W8A8) prefill library, libfp8moe.so.
+ *
+ * The path, in the order the library runs it:
+ *   moe_route        top-k routing with normalised weights, then a stable
+ *                    permutation of (token, slot) pairs by expert;
+ *   moe_quant_act    BF16 rows -> E4M3 codes with one FP32 scale per
+ *                    1x128 group;
+ *   moe_grouped_ffn  grouped gate/up GEMM, unclamped SiLU(gate)*up,
+ *                    requantisation of the intermediate, grouped down GEMM
+ *                    whose epilogue writes routing-weighted FP32 slot rows;
+ *   moe_combine      slot rows summed in slot order, times routed_scaling.
+ *
+ * Sources (web pages, cited by title and section):
+ *   "Full GLM-5.3 streamed FP8 GPU prefill on AVX2 / 2x32GiB SM120",
+ *     section "Design": GPU W8A8 routed experts for prefill (>=256 tokens),
+ *     unclamped SiLU, expert arithmetic tiled at <=4K rows, explicit
+ *     rejection of unsupported dimensions/activation/quantisation, fail
+ *     closed.
+ *   "Integration for GLM-4.6-FP8 and performance tune on H20", gap table
+ *     rows 3, 6, 7: single-wave grid sizing; blockwise FP8 MoE with
+ *     zero-padding of a non-128-divisible intermediate (192 -> 256); fused
+ *     router chain (gate -> top-k -> dispatch).
+ *   "Exact AVX2 FP8 arithmetic conversion avoids costly LUT gathers",
+ *     "Semantics and scope": E4M3 format rules; "Real-checkpoint
+ *     measurements": top-8 routes with normalised routing weights.
+ *   "GLM-5.3-Flash EXL3 on CUDA: a whole prompt pass routes its experts in
+ *     one call", "Exactness" and commit text: one call per pass of up to
+ *     4,096 rows and more, whole-K accumulation without split-K, row bits
+ *     independent of how many rows share the call, routed FP32 rows written
+ *     in place, plan -> grouped gate/up -> grouped down -> combine.
+ *
+ * Conventions for every entry point:
+ *   - Every data pointer is DEVICE memory owned by the caller.  The library
+ *     allocates nothing, keeps no state between calls and never copies or
+ *     repacks weights.  Scratch comes from the caller's workspace, sized by
+ *     the *_workspace_bytes queries.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     only enqueue work; they never synchronise and never read device data
+ *     back to the host, so a sequence of calls can be captured in a CUDA
+ *     graph.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     non-zero moe_status is returned and nothing runs.  There is no CPU
+ *     fallback and no silent fallback.
+ *   - Faults found on the device (an expert id outside [-1, E) in a
+ *     caller-supplied table, a pair index out of range, inconsistent
+ *     offsets, a bounded wait that expired) set bits in a status word at the
+ *     start of that call's workspace; the affected rows are skipped.
+ *     moe_get_device_status reads it.  No kernel traps or spins forever.
+ *   - Layouts are row-major.  Alignment: every pointer 16 bytes.
+ *   - Requires an sm_100 device (B200); other devices get
+ *     MOE_ERR_UNSUPPORTED.
+ */
+#ifndef FP8MOE_H
+#define FP8MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad size, null pointer, out-of-range parameter */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid request this library does not implement */
+    MOE_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+    MOE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than queried */
+    MOE_ERR_CUDA = 5,          /* a CUDA runtime/driver call or launch failed */
+    MOE_ERR_DEVICE_STATUS = 6  /* moe_get_device_status found device-side faults */
+} moe_status;
+
+/* Device status bits (moe_get_device_status). */
+#define MOE_DEV_BAD_EXPERT_ID 0x1  /* an id outside [-1, E) in topk_ids */
+#define MOE_DEV_BAD_PAIR 0x2       /* a sorted_pairs entry outside [0, T*top_k) */
+#define MOE_DEV_BAD_OFFSETS 0x4    /* expert_offsets not monotone or beyond T*top_k */
+#define MOE_DEV_WAIT_TIMEOUT 0x8   /* a bounded wait inside a kernel expired */
+
+/* Limits checked on the host. */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOP_K 32
+#define MOE_MAX_INTERMEDIATE 8192
+#define MOE_MAX_HIDDEN 16384
+
+/* Human-readable name of a moe_status value (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* ABI version of this header, (major << 16) | minor. */
+MOE_API int moe_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- top-k routing and the stable permutation by expert.
+ *
+ * For each token t, the selectable logits (not NaN, not -Inf) are ordered by
+ * value descending, then expert id ascending; the first min(top_k, #selectable)
+ * become the token's slots, in that order.  Slot weights are the softmax of
+ * the selected logits (FP32, expf), so they sum to 1.  Unfilled slots get
+ * id -1 and weight 0.  (Softmax scoring: the tiny workload's statement;
+ * top-k with normalised weights: "Exact AVX2 FP8 arithmetic conversion ...",
+ * "Real-checkpoint measurements".)
+ *
+ * The flat pairs p = t*top_k + j with a valid id are then grouped by expert
+ * with a stable counting sort: expert_offsets[e] is the exclusive prefix of
+ * the per-expert counts (expert_offsets[E] = number of valid pairs, P), and
+ * pair p sits at sorted_pairs[expert_offsets[e] + #{p' < p : id(p') = e}].
+ * Positions P .. T*top_k-1 of sorted_pairs hold -1.  All integer outputs are
+ * deterministic and independent of launch shape.
+ *
+ *   logits          [T, E]      FP32, read
+ *   topk_ids        [T, top_k]  int32, written
+ *   topk_w          [T, top_k]  FP32, written
+ *   expert_offsets  [E + 1]     int32, written
+ *   sorted_pairs    [T * top_k] int32, written
+ *   ws, ws_bytes    scratch of at least moe_route_workspace_bytes(T, E, top_k)
+ *
+ * Limits: T >= 0 (0 is a no-op that still writes expert_offsets = 0),
+ * 1 <= E <= 1024, 0 <= top_k <= min(E, 32).
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_route_workspace_bytes(int64_t T, int E, int top_k);
+MOE_API int moe_route(const float* logits, int64_t T, int E, int top_k,
+              int32_t* topk_ids, float* topk_w,
+              int32_t* expert_offsets, int32_t* sorted_pairs,
+              void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_quant_act -- BF16 activations to E4M3 codes with 1x128 group scales.
+ *
+ * For each token and each group of 128 consecutive columns:
+ *   amax = max |x|;  s = amax / 448 (IEEE FP32 divide);  s == 0 -> s = 1;
+ *   code = E4M3(x / s), round to nearest even, saturating at +-448
+ *   (cvt.rn.satfinite); a group holding NaN or Inf gets s = NaN and every
+ *   code 0x7F.  No flush of subnormals on either side of the divide.
+ * The rule is the plainest reading of W8A8 with per-token 1x128 activation
+ * scales; the pages fix only that activations are FP8 with blockwise scales
+ * ("Integration for GLM-4.6-FP8 ...", row 6; "Full GLM-5.3 ...", "Design").
+ *
+ *   x       [T, H]      BF16 (passed as raw 16-bit words), read
+ *   codes   [T, H]      uint8 E4M3, written
+ *   scales  [T, H/128]  FP32, written
+ *
+ * Limits: T >= 0, H % 128 == 0, 128 <= H <= 16384.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_quant_act(const uint16_t* x, int64_t T, int H,
+                  uint8_t* codes, float* scales, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_ffn -- the experts: grouped gate/up GEMM -> SiLU*up ->
+ * requantise -> grouped down GEMM -> routing-weighted slot rows.
+ *
+ * For every valid pair r (token t, slot j, expert e) taken from
+ * sorted_pairs / expert_offsets:
+ *   g[n] = sum_kb sa[t,kb] * sg[e,n/128,kb] * sum_{k in kb} dec(q[t,k]) dec(Wg[e,n,k])
+ *   u[n] likewise with Wu, su;                         (FP32 accumulation)
+ *   h[n] = g[n] / (1 + exp(-g[n])) * u[n]              (unclamped SiLU)
+ *   (hq, sh) = the moe_quant_act rule applied to h per 128-column group of
+ *              the intermediate (columns I..Ip-1 are zero, Ip = ceil(I/128)*128)
+ *   o[c] = sum_ib sh[ib] * sd[e,c/128,ib] * sum_{i in ib} dec(hq[i]) dec(Wd[e,c,i])
+ *   y[t, j, c] = topk_w[t, j] * o[c]
+ * Rows of y for slots with id -1 are not written.  Each row's bits depend
+ * only on that row's inputs and the expert's weights: no split-K, fixed
+ * K order, tile shapes independent of T ("GLM-5.3-Flash EXL3 on CUDA ...",
+ * "Exactness").  Weights are read in place; a non-128-divisible I is padded
+ * by out-of-bounds zero fill, not by copies ("Integration for GLM-4.6-FP8
+ * ...", row 6).  One call covers all T rows, so each weight tile is streamed
+ * from HBM once per call however large T is ("Full GLM-5.3 ...", "Design":
+ * <=4K-row tiles without repeating the weight transfer).
+ *
+ *   codes, act_scales      [T, H] uint8, [T, H/128] FP32  (moe_quant_act output)
+ *   topk_ids, topk_w       [T, top_k] int32 / FP32        (moe_route output)
+ *   expert_offsets         [E + 1] int32                  (moe_route output)
+ *   sorted_pairs           [T * top_k] int32              (moe_route output)
+ *   w_gate, w_up           [E, I, H] uint8 E4M3 (K-major: each output row contiguous)
+ *   s_gate, s_up           [E, ceil(I/128), H/128] FP32
+ *   w_down                 [E, H, I] uint8 E4M3
+ *   s_down                 [E, H/128, ceil(I/128)] FP32
+ *   y                      [T, top_k, H] FP32, written (valid slots only)
+ *   ws, ws_bytes           scratch of at least moe_ffn_workspace_bytes(T, H, I, E, top_k)
+ *
+ * Limits: H % 128 == 0, 128 <= H <= 16384; I % 16 == 0, 16 <= I <= 8192;
+ * 1 <= E <= 1024; 1 <= top_k <= min(E, 32); T >= 0.  Weight and scale
+ * bytes 0x7F/0xFF (E4M3 NaN) are outside the contract.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ffn_workspace_bytes(int64_t T, int H, int I, int E, int top_k);
+MOE_API int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, int H,
+                    const int32_t* topk_ids, const float* topk_w, int top_k,
+                    const int32_t* expert_offsets, const int32_t* sorted_pairs,
+                    int E, int I,
+                    const uint8_t* w_gate, const float* s_gate,
+                    const uint8_t* w_up, const float* s_up,
+                    const uint8_t* w_down, const float* s_down,
+                    float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- out[t, :] = routed_scaling * sum_{j : id(t,j) >= 0} y[t, j, :]
+ *
+ * Summed in FP32 in slot order j = 0 .. top_k-1 (no atomics), then scaled:
+ * routed scaling is kept with the routed-expert sum ("Full GLM-5.3 ...",
+ * "Design"), and the rows are FP32 ("GLM-5.3-Flash EXL3 on CUDA ...",
+ * commit text).  A token with no valid slot gets exact zeros.  out_bf16,
+ * when not NULL, receives the round-to-nearest-even BF16 of out_f32.
+ *
+ *   y          [T, top_k, H] FP32, read (rows of valid slots)
+ *   topk_ids   [T, top_k] int32, read
+ *   out_f32    [T, H] FP32, written
+ *   out_bf16   [T, H] BF16 words, written, nullable
+ *   ws, ws_bytes  at least moe_combine_workspace_bytes() (status word)
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_combine_workspace_bytes(void);
+MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int H, int top_k, int E,
+                float routed_scaling, float* out_f32, uint16_t* out_bf16,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_get_device_status -- synchronously read the
+ * status word at the start of a workspace used by moe_route,
+ * moe_grouped_ffn or moe_combine.  Waits for all work on the device.
+ * *status_out receives the OR of the MOE_DEV_* bits seen since the last
+ * call on that workspace started; returns MOE_OK, or MOE_ERR_CUDA.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_get_device_status(const void* ws, int* status_out);
+
+/* ---------------------------------------------------------------------------
+ * Test hooks (no counterpart on the pages): the E4M3 encoder and the group
+ * quantiser exactly as the kernels run them, over n device values.
+ *   moe_debug_encode: in[n] FP32 -> out[n] uint8 (cvt.rn.satfinite.e4m3x2).
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8MOE_H */

@@ -1,0 +1,181 @@
+"""GPU parity of the whole layer (route -> quantise -> grouped FFN ->
+combine) against the oracle, at sizes the oracle finishes in seconds (every
+output element) and at the full workload sizes (sampled tokens); row
+invariance, determinism, NaN isolation, degenerate cases and device-side
+fault reporting."""
+import numpy as np
+import pytest
+import torch
+
+import fp8_blockwise_routed_b200 as fm
+import moe_inputs as mi
+from gpu_helpers import assert_close_rows, inputs, oracle_layer, run_layer, sha, tok_rel
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": mi.WORKLOADS["tiny"],
+    # intermediate 192 zero-padded to 256, odd T
+    "i192": mi.Workload("i192", 40, 384, 5, 3, 192, 1.5, "normal", "normal"),
+    # several 128-row tiles per expert with ragged tails; three N tiles
+    "tiles": mi.Workload("tiles", 700, 512, 4, 2, 384, 1.0, "normal_outliers", "normal"),
+    # hidden not a multiple of 256 (half-empty last down tile), I=320
+    "h640": mi.Workload("h640", 333, 640, 12, 4, 320, 0.5, "normal", "uniform"),
+    # one expert, top-1: a dense FFN
+    "dense": mi.Workload("dense", 150, 256, 1, 1, 256, 1.0, "normal", "normal"),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small_every_element(name):
+    wl = SMALL[name]
+    d, h = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    assert layer.device_status() == 0
+    ref = oracle_layer(wl, h)
+    assert np.array_equal(layer.ids[: wl.T].cpu().numpy(), ref["ids"])
+    assert np.array_equal(layer.codes[: wl.T].cpu().numpy(), ref["codes"])
+    assert_close_rows(out, ref["out"])
+    assert np.median(tok_rel(out.double().cpu().numpy(), ref["out"])) < 2e-2
+
+
+@pytest.mark.parametrize("name", ["small", "non128"])
+def test_layer_workload_every_element(name):
+    wl = mi.WORKLOADS[name]
+    d, h = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    assert layer.device_status() == 0
+    ref = oracle_layer(wl, h)
+    assert_close_rows(out, ref["out"])
+
+
+@pytest.mark.parametrize("name", ["glm", "long"])
+def test_layer_workload_sampled(name):
+    """Full-size call; the oracle evaluates a deterministic token sample (all
+    outlier tokens, 256 seeded tokens, tokens of the most and least loaded
+    experts)."""
+    wl = mi.WORKLOADS[name]
+    d, h = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    assert layer.device_status() == 0
+    ids = layer.ids[: wl.T].cpu()
+    toks = mi.sample_tokens(wl, ids).numpy()
+    ref = oracle_layer(wl, h, tokens=toks)
+    assert np.array_equal(ids.numpy(), ref["ids"])
+    assert_close_rows(out, ref["out"], rows=toks)
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiles", "h640"])
+def test_row_invariance(name):
+    """A row's output bits do not depend on how many rows share the call:
+    one call, calls over chunks of rows, and single rows."""
+    wl = SMALL[name]
+    d, _ = inputs(wl)
+    _, full, _ = run_layer(wl, d)
+    full = full.clone()
+    chunk = 37
+    parts = []
+    for t0 in range(0, wl.T, chunk):
+        dd = dict(d, x=d["x"][t0:t0 + chunk].contiguous(), logits=d["logits"][t0:t0 + chunk].contiguous())
+        parts.append(run_layer(wl, dd)[1].clone())
+    assert torch.equal(torch.cat(parts), full)
+    for t in sorted({0, 1, wl.T // 2, wl.T - 1}):
+        dd = dict(d, x=d["x"][t:t + 1].contiguous(), logits=d["logits"][t:t + 1].contiguous())
+        assert torch.equal(run_layer(wl, dd)[1][0], full[t])
+
+
+def test_row_invariance_4096_tiles():
+    """The long-prefill statement: rows give the same bits whether a pass of
+    8,192 rows runs as one call or as two 4,096-row calls."""
+    wl = mi.WORKLOADS["small"].with_(T=8192)
+    d, _ = inputs(wl, seed=1)
+    _, full, _ = run_layer(wl, d)
+    full = full.clone()
+    for t0 in (0, 4096):
+        dd = dict(d, x=d["x"][t0:t0 + 4096].contiguous(), logits=d["logits"][t0:t0 + 4096].contiguous())
+        assert torch.equal(run_layer(wl, dd)[1], full[t0:t0 + 4096])
+
+
+def test_determinism_hashes():
+    wl = SMALL["tiles"]
+    d, _ = inputs(wl)
+    layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"],
+                         wl.k, wl.routed_scaling, wl.T)
+    hashes = set()
+    for _ in range(5):
+        out = layer.forward(d["x"], d["logits"])
+        torch.cuda.synchronize()
+        hashes.add((sha(out), sha(layer.ids[: wl.T]), sha(layer.sorted[: wl.T * wl.k])))
+    assert len(hashes) == 1
+
+
+def test_nan_stays_in_its_row():
+    wl = SMALL["tiles"]
+    d, _ = inputs(wl)
+    _, base, _ = run_layer(wl, d)
+    base = base.clone()
+    x = d["x"].clone()
+    x[17, 3] = float("nan")
+    _, out, _ = run_layer(wl, dict(d, x=x))
+    assert torch.isnan(out[17]).all()
+    keep = torch.ones(wl.T, dtype=torch.bool, device="cuda")
+    keep[17] = False
+    assert torch.equal(out[keep], base[keep])
+
+
+def test_degenerate_cases():
+    wl = SMALL["i192"]
+    d, h = inputs(wl)
+    lg = d["logits"].clone()
+    lg[4] = float("-inf")  # routed to no expert
+    dd = dict(d, logits=lg)
+    _, o1, b1 = run_layer(wl, dd, routed_scaling=1.0, bf16=True)
+    o1 = o1.clone()
+    _, o2, _ = run_layer(wl, dd, routed_scaling=2.0)
+    assert torch.all(o1[4] == 0)
+    assert torch.equal(o2, 2 * o1)
+    assert torch.equal(b1, o1.to(torch.bfloat16))
+    # T = 0
+    d0 = dict(d, x=d["x"][:0], logits=d["logits"][:0])
+    _, o0, _ = run_layer(wl, d0)
+    assert o0.shape == (0, wl.H)
+
+
+def test_experts_without_tokens():
+    """Experts that receive no pairs (the non-128 workload masks 20%) and
+    experts whose only tile is mostly padding."""
+    wl = mi.WORKLOADS["non128"].with_(T=200)
+    d, h = inputs(wl, seed=3)
+    layer, out, _ = run_layer(wl, d)
+    off = layer.offsets.cpu().numpy()
+    masked = mi.masked_experts(wl, 3).numpy()
+    assert np.all(np.diff(off)[masked] == 0)
+    ref = oracle_layer(wl, h)
+    assert_close_rows(out, ref["out"])
+
+
+def test_device_status_bad_ids():
+    wl = SMALL["tiny"]
+    d, _ = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    ids = layer.ids[: wl.T].clone()
+    ids[3, 0] = wl.E + 5
+    ws = torch.empty((fm.moe_combine_workspace_bytes(),), dtype=torch.uint8, device="cuda")
+    o = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
+    fm.moe_combine(layer.y[: wl.T], ids, wl.E, 1.0, o, None, ws)
+    assert fm.moe_get_device_status(ws) & fm.DEV_BAD_EXPERT_ID
+
+
+def test_device_status_bad_offsets():
+    wl = SMALL["tiny"]
+    d, _ = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    off = layer.offsets.clone()
+    off[2] = off[3] + 5  # not monotone
+    y = torch.zeros_like(layer.y[: wl.T])
+    fm.moe_grouped_ffn(layer.codes[: wl.T], layer.scales[: wl.T], layer.ids[: wl.T], layer.tw[: wl.T], off,
+                       layer.sorted[: wl.T * wl.k], *layer.w, y, layer.ws_ffn)
+    st = fm.moe_get_device_status(layer.ws_ffn)
+    assert st & fm.DEV_BAD_OFFSETS
+    assert not (st & fm.DEV_WAIT_TIMEOUT)
+    assert torch.all(y == 0)
