@@ -1,0 +1,370 @@
+"""Benchmark of the routed-MoE FP8 blockwise (W8A8) prefill layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference] [--workload glm]
+
+One step = one whole layer call (moe_quant_act, moe_route, moe_grouped_ffn,
+moe_combine) over one batch of T tokens, inputs resident in HBM.  Workload:
+the GLM-class layer (T=4096, H=5120, 256 experts, top-8, I=1536, 0.1 %
+outlier tokens x100, Zipf(1.1) routing), the configuration the throughput
+target is stated on.  Multi-GPU (torchrun): every rank runs its own batch on
+its own replica of the weights (weak scaling, no collective on the data
+path); the timed region is bracketed by barriers and the time is the max
+over ranks.
+
+Rank 0 prints one JSON line.  Besides the contract keys it carries:
+  roofline      the dominant kernel (the gate/up grouped GEMM), achieved
+                algorithmic bytes / its event-timed duration vs measured HBM
+                copy bandwidth;
+  cpu_baseline  the oracle (plain C, FP64) timed on a bounded token sample
+                on this host's cores;
+  e2e           the same metric with host buffers: pinned H2D of x and
+                logits, the four calls, D2H of the FP32 output, per step;
+  stages        per-launch-group milliseconds from CUDA events;
+  clocks        nvidia-smi samples taken during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "routed-MoE prefill tokens/s per layer; grouped-GEMM % of B200 FP8 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append({"sm": float(f[2]), "max": float(f[3]), "power": float(f[4]),
+                             "hw": f[6], "hw_thermal": f[7], "sw_thermal": f[8], "sw_power": f[9]})
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                            ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        loaded = [r["sm"] for r in rows if r["power"] > 200] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def gateup_alg_bytes(wl, active: int, P: int) -> float:
+    """Algorithmic bytes of one gate/up launch: gate+up FP8 weights of the
+    active experts and their block scales, the activation codes and scales
+    once, the intermediate codes and scales written."""
+    return (2.0 * wl.I * wl.H * active + 2 * 4.0 * active * wl.GI * wl.GH
+            + wl.T * wl.H + 4.0 * wl.T * wl.GH + P * wl.Ip + 4.0 * P * wl.GI)
+
+
+def cpu_baseline(wl, d, budget_tokens: int | None = None):
+    """The oracle as it stands (plain C, FP64, OpenMP) on a seeded token
+    sample of the same workload, timed on the host.  Returns tokens/s."""
+    import oracle
+
+    n = budget_tokens or 24
+    g = mi.generator(0, "cpu_baseline", "cpu")
+    toks = torch.randperm(wl.T, generator=g)[:n].sort().values
+    x = d["x"][toks.to(d["x"].device)].cpu()
+    lg = d["logits"][toks.to(d["logits"].device)].cpu()
+    W = [d[k].cpu() for k in ("w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down")]
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.moe_layer(x, lg, wl.k, *W, wl.routed_scaling)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} seeded tokens of the {wl.name} workload (quantise, route, FFN, combine), "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    """The oracle timed as the reference arm: each step evaluates a bounded
+    seeded sample of the workload's tokens on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    d = mi.make_inputs(wl, 0, "cpu")
+    n = 8
+    W = [d[k] for k in ("w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down")]
+    oracle.build()
+
+    def step(i):
+        g = mi.generator(i, "reference_sample", "cpu")
+        toks = torch.randperm(wl.T, generator=g)[:n].sort().values
+        oracle.moe_layer(d["x"][toks], d["logits"][toks], wl.k, *W, wl.routed_scaling)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    cores = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n} seeded tokens per step of the {wl.name} workload"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} top_k={wl.k} I={wl.I} "
+                        f"rs={wl.routed_scaling} x={wl.x_dist} logits={wl.logit_dist}",
+            "global_batch": wl.T, "parallelism": "data-parallel replicas (one batch per GPU)",
+            "l2": "inputs larger than L2: FP8 expert weights read per step exceed 126 MB"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default="glm", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    wl = mi.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import fp8_blockwise_routed_b200 as fm
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = mi.make_inputs(wl, seed=rank, device=dev)
+    layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"],
+                         wl.k, wl.routed_scaling, wl.T)
+    s = torch.cuda.current_stream()
+
+    # events: 7 per step (quantise, route, gather, gate/up, down, combine, end)
+    def mk():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(s)
+        return e
+
+    evs = [[mk() for _ in range(7)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        layer.forward(d["x"], d["logits"])
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status reported a fault during warm-up")
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for i in range(args.steps):
+        layer.forward(d["x"], d["logits"], stage_events=evs[i])
+    t1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms_total = max_over_ranks(world, t0.elapsed_time(t1))
+    ms_step = ms_total / args.steps
+    status = layer.device_status()
+    names = ["quant_act", "route", "gather", "gemm_gateup", "gemm_down", "combine"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(names)}
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    off = layer.offsets.cpu()
+    P = int(off[-1])
+    active = int(((off[1:] - off[:-1]) > 0).sum())
+    gu_bytes = gateup_alg_bytes(wl, active, P)
+    gu_s = stage_ms["gemm_gateup"] / 1e3
+    achieved = gu_bytes / gu_s / 1e9
+    flops = mi.flops_per_layer(wl, P)
+    gemm_s = (stage_ms["gemm_gateup"] + stage_ms["gemm_down"]) / 1e3
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal FP8:BF16 ratio 2 on the measured BF16 peak
+    layer_bytes = mi.algorithmic_bytes(wl, active)
+    roof_s = max(flops / (fp8_peak * 1e12), (layer_bytes - wl.T * wl.H * 4 - wl.T * wl.H * 2 - wl.T * wl.E * 4)
+                 / (pk["hbm_gbs"] * 1e9))
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        t = json.load(open(prof)).get(f"gemm_gateup/{wl.name}")
+        traffic = t if t else None
+
+    # end to end through the C ABI with host buffers
+    x_h = d["x"].cpu().pin_memory()
+    lg_h = d["logits"].cpu().pin_memory()
+    out_h = torch.empty((wl.T, wl.H), dtype=torch.float32).pin_memory()
+    x_d = torch.empty_like(d["x"])
+    lg_d = torch.empty_like(d["logits"])
+    for _ in range(2):
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        out_h.copy_(layer.forward(x_d, lg_d), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        out_h.copy_(layer.forward(x_d, lg_d), non_blocking=True)
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, d)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": world * wl.T / (ms_step / 1e3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "fp8e4m3 (fp32 accumulate)",
+            "data": "synthetic (seeded; no checkpoint)",
+            "config": workload_config(wl),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                         "kernel": "grouped_gemm_kernel<gate/up>",
+                         "alg_bytes_per_launch": gu_bytes, "peak_source": pk["source"]},
+            "grouped_gemm": {"ms": gemm_s * 1e3, "tflops": flops / gemm_s / 1e12,
+                             "frac_fp8_peak": flops / gemm_s / 1e12 / fp8_peak,
+                             "fp8_peak_tflops": fp8_peak, "roofline_ms": roof_s * 1e3,
+                             "frac_roofline": roof_s / gemm_s},
+            "stages_ms": stage_ms,
+            "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
+                    "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms},
+            "gpu_launches": 8 * args.steps,
+            "device_status": status,
+            "active_experts": active,
+            "pairs": P,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        if clocks:
+            line["clocks"] = clocks
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -27,8 +27,8 @@ _lib = None
 
 
 class MoeError(RuntimeError):
-    def __init__(self, code: int, what: str):
-        super().__init__(f"{what} failed: {STATUS.get(code, code)}")
+    def __init__(self, code: int, what: str, detail: str = ""):
+        super().__init__(f"{what} failed: {STATUS.get(code, code)}" + (f" ({detail})" if detail else ""))
         self.code = code
 
 
@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i32]
         L.moe_abi_version.restype = i32
+        L.moe_last_error.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = []
         L.moe_route_workspace_bytes.restype = sz
         L.moe_route_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_route.restype = i32
@@ -59,7 +61,7 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
         L.moe_grouped_ffn.restype = i32
         L.moe_grouped_ffn.argtypes = [P, P, i64, i32, P, P, i32, P, P, i32, i32,
-                                      P, P, P, P, P, P, P, P, sz, P]
+                                      P, P, P, P, P, P, P, P, sz, P, P]
         L.moe_combine_workspace_bytes.restype = sz
         L.moe_combine_workspace_bytes.argtypes = []
         L.moe_combine.restype = i32
@@ -88,7 +90,8 @@ def _s(stream):
 
 def _check(code: int, what: str):
     if code != 0:
-        raise MoeError(code, what)
+        detail = lib().moe_last_error().decode() if code in (2, 5) else ""
+        raise MoeError(code, what, detail)
 
 
 # ------------------------------------------------------------------ sizes
@@ -119,14 +122,19 @@ def moe_quant_act(x, codes, scales, stream=None):
 
 
 def moe_grouped_ffn(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs,
-                    w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None):
+                    w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None, stage_events=None):
+    """stage_events: None or 4 torch.cuda.Event objects (already recorded
+    once, so that their handles exist) marking gather / gate-up / down / end."""
     T, H = codes.shape
     E, I, _ = w_gate.shape
     top_k = topk_ids.shape[1]
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * 4)(*[e.cuda_event for e in stage_events])
     _check(lib().moe_grouped_ffn(_p(codes), _p(act_scales), T, H, _p(topk_ids), _p(topk_w), top_k,
                                  _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate),
                                  _p(w_up), _p(s_up), _p(w_down), _p(s_down), _p(y), _p(ws),
-                                 ws.numel() * ws.element_size(), _s(stream)), "moe_grouped_ffn")
+                                 ws.numel() * ws.element_size(), _s(stream), ev), "moe_grouped_ffn")
 
 
 def moe_combine(y, topk_ids, num_experts, routed_scaling, out_f32, out_bf16, ws, stream=None):
@@ -178,16 +186,27 @@ class RoutedMoE:
         self.ws_comb = torch.empty((moe_combine_workspace_bytes(),), dtype=u8, device=dev)
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, out_bf16: torch.Tensor | None = None,
-                stream=None) -> torch.Tensor:
+                stream=None, stage_events=None) -> torch.Tensor:
+        """stage_events: None, or 7 recorded torch.cuda.Events marking the
+        start of quantise, route, gather, gate/up, down, combine and the end."""
         T = x.shape[0]
         assert T <= self.max_tokens and x.shape[1] == self.H and logits.shape == (T, self.E)
         codes, scales = self.codes[:T], self.scales[:T]
         ids, tw, srt = self.ids[:T], self.tw[:T], self.sorted[: T * self.k]
         y, out = self.y[:T], self.out[:T]
+        ev = stage_events
+        s = torch.cuda.current_stream() if stream is None else stream
+        if ev is not None:
+            ev[0].record(s)
         moe_quant_act(x, codes, scales, stream)
+        if ev is not None:
+            ev[1].record(s)
         moe_route(logits, self.k, ids, tw, self.offsets, srt, self.ws_route, stream)
-        moe_grouped_ffn(codes, scales, ids, tw, self.offsets, srt, *self.w, y, self.ws_ffn, stream)
+        moe_grouped_ffn(codes, scales, ids, tw, self.offsets, srt, *self.w, y, self.ws_ffn, stream,
+                        stage_events=None if ev is None else ev[2:6])
         moe_combine(y, ids, self.E, self.rs, out, out_bf16, self.ws_comb, stream)
+        if ev is not None:
+            ev[6].record(s)
         return out
 
     def device_status(self) -> int:

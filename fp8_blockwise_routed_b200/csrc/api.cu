@@ -54,20 +54,34 @@ namespace {
 
 constexpr size_t kStatusBytes = 256;
 
+thread_local char g_last_error[256] = "";
+
+// Record a failed CUDA call for moe_last_error() and map it to a status.
+int cuda_fail(cudaError_t err, const char* where)
+{
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(err),
+                  static_cast<int>(err));
+    return err == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Common device check: an sm_100 GPU must be current.
 int check_device()
 {
     DeviceInfo di;
-    if (!device_info(&di)) return MOE_ERR_CUDA;
+    if (!device_info(&di)) {
+        std::snprintf(g_last_error, sizeof(g_last_error), "no usable CUDA device");
+        return MOE_ERR_CUDA;
+    }
     if (di.major != 10 || di.minor != 0) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
 int clear_status(void* ws, cudaStream_t s)
 {
-    return cudaMemsetAsync(ws, 0, sizeof(int), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const cudaError_t err = cudaMemsetAsync(ws, 0, sizeof(int), s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "status clear");
 }
 
 size_t route_layout(int64_t T, int E, int k, size_t* off_hist, size_t* off_rank)
@@ -101,6 +115,8 @@ const char* moe_status_string(int status)
 
 int moe_abi_version(void) { return (1 << 16) | 0; }
 
+const char* moe_last_error(void) { return g_last_error; }
+
 size_t moe_route_workspace_bytes(int64_t T, int E, int top_k)
 {
     if (T < 0 || E < 1 || top_k < 0) return 0;
@@ -128,7 +144,7 @@ int moe_route(const float* logits, int64_t T, int E, int top_k, int32_t* topk_id
     cudaError_t err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
                                    reinterpret_cast<int32_t*>(w8 + off_hist), reinterpret_cast<int32_t*>(w8 + off_rank),
                                    s);
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route");
 }
 
 int moe_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* scales, void* stream)
@@ -139,7 +155,7 @@ int moe_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* sc
     if (T == 0) return MOE_OK;
     if (int r = check_device()) return r;
     cudaError_t err = launch_quant_act(x, T, H, codes, scales, static_cast<cudaStream_t>(stream));
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quant_act");
 }
 
 size_t moe_ffn_workspace_bytes(int64_t T, int H, int I, int E, int top_k)
@@ -154,7 +170,7 @@ int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, in
                     const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs,
                     int E, int I, const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
                     const float* s_up, const uint8_t* w_down, const float* s_down, float* y, void* ws,
-                    size_t ws_bytes, void* stream)
+                    size_t ws_bytes, void* stream, void* const* stage_events)
 {
     if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOP_K) return MOE_ERR_INVALID_ARG;
@@ -200,9 +216,9 @@ int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, in
     a.sa_sorted = reinterpret_cast<float*>(w8 + off_sa);
     a.h_codes = w8 + off_h;
     a.h_scales = reinterpret_cast<float*>(w8 + off_sh);
+    a.stage_events = stage_events;
     cudaError_t err = launch_grouped_ffn(a, s);
-    if (err == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_ffn");
 }
 
 size_t moe_combine_workspace_bytes(void) { return kStatusBytes; }
@@ -221,15 +237,17 @@ int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int H, int t
     if (int r = clear_status(ws, s)) return r;
     cudaError_t err = launch_combine(y, topk_ids, T, H, top_k, E, routed_scaling, out_f32, out_bf16,
                                      static_cast<int*>(ws), s);
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
 }
 
 int moe_get_device_status(const void* ws, int* status_out)
 {
     if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
-    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t err = cudaDeviceSynchronize();
+    if (err != cudaSuccess) return cuda_fail(err, "moe_get_device_status sync");
     int v = 0;
-    if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    err = cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_get_device_status copy");
     *status_out = v;
     return MOE_OK;
 }
@@ -239,7 +257,7 @@ int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* stream)
     if (n < 0 || (n > 0 && (!in || !out))) return MOE_ERR_INVALID_ARG;
     if (int r = check_device()) return r;
     cudaError_t err = launch_encode(in, n, out, static_cast<cudaStream_t>(stream));
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_encode");
 }
 
 }  // extern "C"

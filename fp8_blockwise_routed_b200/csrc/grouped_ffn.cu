@@ -25,15 +25,15 @@
 // Two partial buffers of 256 TMEM columns alternate, so the MMA of block kb+1
 // overlaps the promotion of block kb.
 //
-// Warp roles (320 threads, one CTA per SM, grid = #SMs, static round-robin
+// Warp roles (384 threads, one CTA per SM, grid = #SMs, static round-robin
 // over work items ordered expert-major, then n-tile, then m-tile so that the
 // m-tiles sharing a weight panel run at the same time and share it in L2):
 //   warp 0      TMA producer (one lane): A tile 128x128 B, B tile 2x128x128 B
 //               per stage, 4 stages, mbarrier complete_tx
-//   warp 1      TMEM allocator and MMA issuer (one lane)
-//   warps 2..9  promotion + epilogue; warp w reads TMEM lanes 32*(w%4) (its
-//               rows); warps 2..5 own columns [0,64) of each 128-half, warps
-//               6..9 columns [64,128)
+//   warp 1      TMEM allocator and MMA issuer (one lane); warps 2-3 idle
+//   warps 4..11 promotion + epilogue; warp w reads TMEM lanes 32*(w%4) (its
+//               rows); warps 4..7 own columns [0,64) of each 128-half, warps
+//               8..11 columns [64,128)
 // Every wait is bounded (2 s of global time); on expiry the CTA raises an
 // abort flag, records MOE_DEV_WAIT_TIMEOUT, drains and frees TMEM.
 #include <cuda.h>
@@ -58,7 +58,16 @@ constexpr int A_TILE = BM * BK;           // 16 KiB
 constexpr int B_HALF = 128 * BK;          // 16 KiB
 constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int THREADS = 128 + EPI_WARPS * 32;  // 3 warpgroups
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64,512);
+// the producer/MMA warpgroup drops to 40 and the two epilogue warpgroups rise
+// to 232: 128 x 40 + 256 x 232 = 64,512, the launch total.  Each SM
+// sub-partition holds one warp of each warpgroup:
+// 32 x (40 + 232 + 232) = 16,128 <= 16,384 registers.
+constexpr uint32_t REGS_CTRL = 40;
+constexpr uint32_t REGS_EPI = 232;
+static_assert(128 * REGS_CTRL + 256 * REGS_EPI <= THREADS * 168, "register split exceeds the launch budget");
+static_assert(32 * (REGS_CTRL + 2 * REGS_EPI) <= 16384, "register split exceeds a sub-partition");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr int MAX_E = 1024;
@@ -125,7 +134,7 @@ __device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int
 // ---------------------------------------------------------------- roles
 
 template <int MODE>
-__device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB0, const CUtensorMap* tmB1,
+__device__ __forceinline__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB0, const CUtensorMap* tmB1,
                               const GemmParams& p, const int* seg, const int* ipre, int total_items,
                               uint32_t sbase, uint32_t bars, volatile int* abort)
 {
@@ -162,7 +171,7 @@ __device__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB0, c
     }
 }
 
-__device__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars, uint32_t tmem,
+__device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort)
 {
     const int lane = threadIdx.x & 31;
@@ -207,13 +216,13 @@ drain:
 }
 
 template <int MODE>
-__device__ void epilogue_role(const GemmParams& p, const int* seg, const int* ipre, int total_items, uint32_t bars,
+__device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* seg, const int* ipre, int total_items, uint32_t bars,
                               uint32_t tmem, float* amax_x, volatile int* abort)
 {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;        // column half-slice of each 128-wide half
+    const int half = (warp - 4) >> 2;        // column half-slice of each 128-wide half
     const int trow = q * 32 + lane;          // row within the tile
     const uint32_t tfull0 = bars + 2 * STAGES * 8, tempty0 = tfull0 + 16, xbar0 = tempty0 + 16;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -351,7 +360,7 @@ __device__ void epilogue_role(const GemmParams& p, const int* seg, const int* ip
 }
 
 template <int MODE>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const GemmParams p)
 {
@@ -416,12 +425,16 @@ __global__ void __maxnreg__(200)
     const uint32_t tmem = *tmem_slot;
     const int total_items = *bad ? 0 : ipre[E];
 
-    if (warp == 0) {
-        if ((threadIdx.x & 31) == 0)
-            producer_role<MODE>(&tmA, &tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
-    } else if (warp == 1) {
-        mma_role(p, total_items, sbase, bars, tmem, abort);
+    if (warp < 4) {
+        setmaxnreg_dec<REGS_CTRL>();
+        if (warp == 0) {
+            if ((threadIdx.x & 31) == 0)
+                producer_role<MODE>(&tmA, &tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
+        } else if (warp == 1) {
+            mma_role(p, total_items, sbase, bars, tmem, abort);
+        }
     } else {
+        setmaxnreg_inc<REGS_EPI>();
         epilogue_role<MODE>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
     }
 
@@ -540,6 +553,14 @@ size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_
     return o;
 }
 
+namespace {
+cudaError_t stage_mark(const FfnArgs& a, int i, cudaStream_t s)
+{
+    if (!a.stage_events || !a.stage_events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(a.stage_events[i]), s);
+}
+}  // namespace
+
 cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
 {
     const int64_t P = a.T * a.k;
@@ -550,6 +571,8 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     const int H = a.H, I = a.I, E = a.E;
     const int GH = H / 128, GI = (I + 127) / 128, Ip = GI * 128;
 
+    cudaError_t err = stage_mark(a, 0, s);
+    if (err != cudaSuccess) return err;
     // 1. gather the A operand rows (and their scales) into expert order
     {
         const int64_t want = ceil_div64(P, 8);
@@ -557,7 +580,7 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
         gather_rows_kernel<<<static_cast<int>(want < cap ? want : cap), 256, 0, s>>>(
             a.codes, a.act_scales, H, a.k, a.sorted_pairs, a.expert_offsets, E, P, a.a_sorted, a.sa_sorted,
             a.status);
-        cudaError_t err = cudaGetLastError();
+        err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
 
@@ -599,7 +622,8 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     g.y = a.y;
     g.H = H;
     g.status = a.status;
-    cudaError_t err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
+    if ((err = stage_mark(a, 1, s)) != cudaSuccess) return err;
+    err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
     if (err != cudaSuccess) return err;
 
     // 4. down GEMM with the routing-weighted row epilogue
@@ -610,7 +634,9 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     d.b_s0 = a.s_down;
     d.b_s1 = a.s_down;
     d.b_nblocks = GH;
-    return run_gemm<1>(tmA2, tmD, tmD, d, grid, s);
+    if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
+    if ((err = run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;
+    return stage_mark(a, 3, s);
 }
 
 }  // namespace fp8moe

@@ -63,6 +63,7 @@ struct FfnArgs {
     float* sa_sorted;    // [P, H/128]
     uint8_t* h_codes;    // [P, Ip]
     float* h_scales;     // [P, ceil(I/128)]
+    void* const* stage_events;  // nullable: 4 cudaEvent_t for profiling
 };
 size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
                             size_t* off_sh);

@@ -96,6 +96,11 @@ MOE_API const char* moe_status_string(int status);
 /* ABI version of this header, (major << 16) | minor. */
 MOE_API int moe_abi_version(void);
 
+/* Text of the last CUDA failure seen by this thread in a call that returned
+ * MOE_ERR_CUDA or MOE_ERR_UNSUPPORTED from the device ("" if none).  The
+ * string is owned by the library and valid until the thread's next call. */
+MOE_API const char* moe_last_error(void);
+
 /* ---------------------------------------------------------------------------
  * moe_route -- top-k routing and the stable permutation by expert.
  *
@@ -183,6 +188,10 @@ MOE_API int moe_quant_act(const uint16_t* x, int64_t T, int H,
  *   s_down                 [E, H/128, ceil(I/128)] FP32
  *   y                      [T, top_k, H] FP32, written (valid slots only)
  *   ws, ws_bytes           scratch of at least moe_ffn_workspace_bytes(T, H, I, E, top_k)
+ *   stage_events           NULL, or 4 cudaEvent_t handles for profiling: event i
+ *                          is recorded on `stream` before stage i (0 = gather of
+ *                          the A rows, 1 = gate/up GEMM, 2 = down GEMM) and event
+ *                          3 after the down GEMM.  Owned by the caller.
  *
  * Limits: H % 128 == 0, 128 <= H <= 16384; I % 16 == 0, 16 <= I <= 8192;
  * 1 <= E <= 1024; 1 <= top_k <= min(E, 32); T >= 0.  Weight and scale
@@ -196,7 +205,8 @@ MOE_API int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64
                     const uint8_t* w_gate, const float* s_gate,
                     const uint8_t* w_up, const float* s_up,
                     const uint8_t* w_down, const float* s_down,
-                    float* y, void* ws, size_t ws_bytes, void* stream);
+                    float* y, void* ws, size_t ws_bytes, void* stream,
+                    void* const* stage_events);
 
 /* ---------------------------------------------------------------------------
  * moe_combine -- out[t, :] = routed_scaling * sum_{j : id(t,j) >= 0} y[t, j, :]

@@ -67,7 +67,7 @@ def test_quant_validation(L):
 def _ffn(L, T=4, H=256, k=2, E=8, I=128, ws=None, ptr=A):
     if ws is None:
         ws = L.moe_ffn_workspace_bytes(T, H, I, E, k)
-    return L.moe_grouped_ffn(ptr, A, T, H, A, A, k, A, A, E, I, A, A, A, A, A, A, A, A, ws, None)
+    return L.moe_grouped_ffn(ptr, A, T, H, A, A, k, A, A, E, I, A, A, A, A, A, A, A, A, ws, None, None)
 
 
 def test_ffn_validation(L):
