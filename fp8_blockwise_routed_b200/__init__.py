@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.moe_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         L.moe_debug_encode.restype = i32
         L.moe_debug_encode.argtypes = [P, i64, P, P]
+        L.moe_ffn_intermediate.restype = i32
+        L.moe_ffn_intermediate.argtypes = [P, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p),
+                                           ctypes.POINTER(ctypes.c_void_p)]
         _lib = L
     return _lib
 
@@ -153,6 +156,22 @@ def moe_get_device_status(ws) -> int:
 
 def moe_debug_encode(inp, out, stream=None):
     _check(lib().moe_debug_encode(_p(inp), inp.numel(), _p(out), _s(stream)), "moe_debug_encode")
+
+
+def moe_ffn_intermediate(ws, T: int, H: int, I: int, top_k: int):
+    """(codes [T*top_k, Ip] uint8, scales [T*top_k, ceil(I/128)] float32)
+    views of the intermediate held in a grouped-FFN workspace, rows in
+    expert order."""
+    c, sc = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib().moe_ffn_intermediate(_p(ws), T, H, I, top_k, ctypes.byref(c), ctypes.byref(sc)),
+           "moe_ffn_intermediate")
+    GI = (I + 127) // 128
+    base = ws.data_ptr()
+    oc, osc = c.value - base, sc.value - base
+    P = T * top_k
+    codes = ws[oc: oc + P * GI * 128].view(P, GI * 128)
+    scales = ws[osc: osc + P * GI * 4].view(torch.float32).view(P, GI)
+    return codes, scales
 
 
 # ------------------------------------------------------------------ layer

@@ -260,4 +260,15 @@ int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* stream)
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_encode");
 }
 
+int moe_ffn_intermediate(const void* ws, int64_t T, int H, int I, int top_k, const uint8_t** h_codes,
+                         const float** h_scales)
+{
+    if (!ws || !h_codes || !h_scales || T < 0 || H < 128 || I < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
+    size_t off_a, off_sa, off_h, off_sh;
+    ffn_workspace_layout(T, H, I, top_k, &off_a, &off_sa, &off_h, &off_sh);
+    *h_codes = static_cast<const uint8_t*>(ws) + off_h;
+    *h_scales = reinterpret_cast<const float*>(static_cast<const uint8_t*>(ws) + off_sh);
+    return MOE_OK;
+}
+
 }  // extern "C"

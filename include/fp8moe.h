@@ -238,11 +238,19 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
 MOE_API int moe_get_device_status(const void* ws, int* status_out);
 
 /* ---------------------------------------------------------------------------
- * Test hooks (no counterpart on the pages): the E4M3 encoder and the group
- * quantiser exactly as the kernels run them, over n device values.
- *   moe_debug_encode: in[n] FP32 -> out[n] uint8 (cvt.rn.satfinite.e4m3x2).
+ * Test hooks (no counterpart on the pages).
+ *   moe_debug_encode: in[n] FP32 -> out[n] uint8 E4M3, the encoder the
+ *   kernels use (cvt.rn.satfinite.e4m3x2).
  * ------------------------------------------------------------------------- */
 MOE_API int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* stream);
+
+/* moe_ffn_intermediate: device pointers into a workspace last used by
+ * moe_grouped_ffn with the same (T, H, I, top_k): the requantised
+ * intermediate codes [T*top_k, Ip] and their scales [T*top_k, ceil(I/128)],
+ * rows in expert order (row r belongs to pair sorted_pairs[r]).  Host
+ * arithmetic only; nothing is read from the device. */
+MOE_API int moe_ffn_intermediate(const void* ws, int64_t T, int H, int I, int top_k,
+                                 const uint8_t** h_codes, const float** h_scales);
 
 #ifdef __cplusplus
 }

@@ -56,7 +56,7 @@ def open_library(path: str) -> ctypes.CDLL:
     lib.oracle_permute.argtypes = [P, i64, i32, i32, P, P]
     lib.oracle_moe_ffn.argtypes = [P, P, i64, i64, P, P, i32, i32, i64,
                                    P, P, P, P, P, P, ctypes.c_double,
-                                   P, i64, P, P, P, P, P, P, i32]
+                                   P, i64, P, P, P, P, P, P, P, i32]
     lib.oracle_num_threads.restype = i32
     return lib
 
@@ -191,7 +191,7 @@ def moe_ffn(codes, act_scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_dow
 
     Returns a dict with ``out`` float64 [n,H] and, on request, ``slots``
     float64 [n,k,H] (w_j * o_j), ``h_codes`` uint8 [n,k,Ip], ``h_scales``
-    float32 [n,k,G_I].  ``h_override=(codes, scales)`` in that layout replaces
+    float32 [n,k,G_I] and ``h_fp32`` float32 [n,k,Ip] (h before requantisation).  ``h_override=(codes, scales)`` in that layout replaces
     the intermediate used by the down projection.
     """
     codes = _np(codes, np.uint8)
@@ -215,6 +215,7 @@ def moe_ffn(codes, act_scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_dow
     slots = np.zeros((n, k, H), np.float64) if want_slots else None
     hc = np.zeros((n, k, Ip), np.uint8) if want_h else None
     hs = np.zeros((n, k, GI), np.float32) if want_h else None
+    hf = np.zeros((n, k, Ip), np.float32) if want_h else None
     oc = os_ = None
     if h_override is not None:
         oc = np.ascontiguousarray(h_override[0], dtype=np.uint8)
@@ -223,12 +224,12 @@ def moe_ffn(codes, act_scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_dow
     _load().oracle_moe_ffn(_ptr(codes), _ptr(act_scales), T, H, _ptr(ids), _ptr(w), k, E, I,
                            _ptr(wg), _ptr(sg), _ptr(wu), _ptr(su), _ptr(wd), _ptr(sd),
                            float(routed_scaling), _ptr(tokens), n, _ptr(out), _ptr(slots),
-                           _ptr(hc), _ptr(hs), _ptr(oc), _ptr(os_), int(n_threads))
+                           _ptr(hc), _ptr(hs), _ptr(hf), _ptr(oc), _ptr(os_), int(n_threads))
     res = {"out": out}
     if want_slots:
         res["slots"] = slots
     if want_h:
-        res["h_codes"], res["h_scales"] = hc, hs
+        res["h_codes"], res["h_scales"], res["h_fp32"] = hc, hs, hf
     return res
 
 

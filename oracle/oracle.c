@@ -228,7 +228,8 @@ ORACLE_API void oracle_permute(const int32_t* ids, int64_t T, int k, int E,
 /*   wd [E,H,I];     sd [E,H/128,ceil(I/128)]      down weights+scales       */
 /*   out [n_tok,H] FP64                            routed output rows        */
 /*   slot_out [n_tok,k,H] FP64 (nullable)          w_j * o_j per slot        */
-/*   h_codes [n_tok,k,Ip], h_scales [n_tok,k,G_I] (nullable) intermediate    */
+/*   h_codes [n_tok,k,Ip], h_scales [n_tok,k,G_I] (nullable) intermediate;   */
+/*   h_fp32 [n_tok,k,Ip] (nullable) the FP32 h before requantisation         */
 /*   h_override_codes/h_override_scales (nullable): same layout as h_codes;  */
 /*     when given, the down projection uses them instead of its own (used to */
 /*     isolate the down-projection error of another implementation).         */
@@ -244,7 +245,7 @@ ORACLE_API void oracle_moe_ffn(const uint8_t* codes, const float* act_scales,
                                double routed_scaling,
                                const int64_t* token_list, int64_t n_tok,
                                double* out, double* slot_out,
-                               uint8_t* h_codes, float* h_scales,
+                               uint8_t* h_codes, float* h_scales, float* h_fp32,
                                const uint8_t* h_override_codes,
                                const float* h_override_scales,
                                int n_threads)
@@ -312,6 +313,10 @@ ORACLE_API void oracle_moe_ffn(const uint8_t* codes, const float* act_scales,
                     int64_t c0 = gi * 128;
                     int64_t nc = (I - c0 < 128) ? (I - c0) : 128;
                     oracle_quant_group(h32 + c0, (int)nc, hq + c0, sh + gi);
+                }
+                if (h_fp32) {
+                    memcpy(h_fp32 + (it * k + j) * Ip, h32, (size_t)I * sizeof(float));
+                    for (int64_t n = I; n < Ip; ++n) h_fp32[(it * k + j) * Ip + n] = 0.0f;
                 }
                 if (h_codes) memcpy(h_codes + (it * k + j) * Ip, hq, (size_t)Ip);
                 if (h_scales) memcpy(h_scales + (it * k + j) * GI, sh, (size_t)GI * sizeof(float));
