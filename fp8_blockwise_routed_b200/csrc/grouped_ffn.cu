@@ -251,30 +251,40 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             acc0[i] = 0.f;
             acc1[i] = 0.f;
         }
-        float sa_next = __ldg(sa_row);
+        // scales of K block kb+1 are fetched while block kb is promoted
+        float sa_n = __ldg(sa_row), w0_n = __ldg(s0), w1_n = has1 ? __ldg(s1) : 0.f;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             const int b = it & 1;
             const uint32_t bph = (it >> 1) & 1;
-            const float sa = sa_next;
-            if (kb + 1 < p.num_kb) sa_next = __ldg(sa_row + kb + 1);
-            const float c0 = sa * __ldg(s0 + kb);
-            const float c1 = has1 ? sa * __ldg(s1 + kb) : 0.f;
+            const float c0 = sa_n * w0_n;
+            const float c1 = sa_n * w1_n;
+            if (kb + 1 < p.num_kb) {
+                sa_n = __ldg(sa_row + kb + 1);
+                w0_n = __ldg(s0 + kb + 1);
+                if (has1) w1_n = __ldg(s1 + kb + 1);
+            }
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, bph, abort, WAIT_NS))) return;
             tc_fence_after();
             const uint32_t col = lane_base + b * 256 + half * 64;
-            float v[32];
-            tmem_ld32(col, v);
+            // four 32-column loads; each load after the first overlaps the
+            // FMAs of the one before
+            uint32_t ra[32], rb[32];
+            tmem_ld32_issue(col, ra);
+            tmem_ld_wait(ra);
+            tmem_ld32_issue(col + 32, rb);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc0[i] = fmaf(c0, v[i], acc0[i]);
-            tmem_ld32(col + 32, v);
+            for (int i = 0; i < 32; ++i) acc0[i] = fmaf(c0, __uint_as_float(ra[i]), acc0[i]);
+            tmem_ld_wait(rb);
+            tmem_ld32_issue(col + 128, ra);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc0[32 + i] = fmaf(c0, v[i], acc0[32 + i]);
-            tmem_ld32(col + 128, v);
+            for (int i = 0; i < 32; ++i) acc0[32 + i] = fmaf(c0, __uint_as_float(rb[i]), acc0[32 + i]);
+            tmem_ld_wait(ra);
+            tmem_ld32_issue(col + 160, rb);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc1[i] = fmaf(c1, v[i], acc1[i]);
-            tmem_ld32(col + 160, v);
+            for (int i = 0; i < 32; ++i) acc1[i] = fmaf(c1, __uint_as_float(ra[i]), acc1[i]);
+            tmem_ld_wait(rb);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(c1, v[i], acc1[32 + i]);
+            for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(c1, __uint_as_float(rb[i]), acc1[32 + i]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty0 + 8 * b);
@@ -290,7 +300,9 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 const float g = acc0[i];
-                const float h = __fdiv_rn(g, 1.0f + expf(-g)) * acc1[i];
+                // SiLU(g) = g / (1 + exp(-g)), as g times the correctly
+                // rounded reciprocal (within 1.5 ulp of the quotient)
+                const float h = g * __frcp_rn(1.0f + expf(-g)) * acc1[i];
                 acc0[i] = h;
                 if (isfinite(h)) amax = fmaxf(amax, fabsf(h));
                 else bad = 1;
@@ -314,15 +326,24 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
 #pragma unroll
                     for (int c = 0; c < 4; ++c) reinterpret_cast<uint4*>(dst)[c] = nanq;
                 } else {
+                    // h / s as h times the correctly rounded reciprocal of s
+                    // (within 1 ulp of the quotient; a code can differ from
+                    // the divide's only when h/s lies within that ulp of an
+                    // E4M3 rounding boundary).  Scales whose reciprocal
+                    // overflows use the divide.
+                    const float inv = __frcp_rn(s);
+                    const bool use_div = !isfinite(inv);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t wv[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int i = c * 16 + j * 4;
-                            const uint32_t lo = e4m3x2(__fdiv_rn(acc0[i], s), __fdiv_rn(acc0[i + 1], s));
-                            const uint32_t hi = e4m3x2(__fdiv_rn(acc0[i + 2], s), __fdiv_rn(acc0[i + 3], s));
-                            wv[j] = lo | (hi << 16);
+                            float q[4];
+#pragma unroll
+                            for (int m = 0; m < 4; ++m)
+                                q[m] = use_div ? __fdiv_rn(acc0[i + m], s) : acc0[i + m] * inv;
+                            wv[j] = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
                         }
                         reinterpret_cast<uint4*>(dst)[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                     }

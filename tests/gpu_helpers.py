@@ -115,7 +115,7 @@ def gpu_intermediate_by_pair(layer, T: int):
     return gc.reshape(T, k, Ip), gs.reshape(T, k, GI)
 
 
-def check_layer(wl, layer, gpu_out, ref, h, tokens=None, mid_tol=0.05):
+def check_layer(wl, layer, gpu_out, ref, h, tokens=None, mid_tol=1e-4):
     """Full comparison of a layer call with the oracle (``ref`` computed with
     want_h=True for ``tokens``, default all).  Returns a dict of statistics."""
     T = gpu_out.shape[0]
@@ -148,14 +148,17 @@ def check_layer(wl, layer, gpu_out, ref, h, tokens=None, mid_tol=0.05):
         t_i, j_i, c_i = np.nonzero(flips)
         r_g = rank[gc[t_i, j_i, c_i]]
         r_o = rank[oc[t_i, j_i, c_i]]
-        assert np.all(np.abs(r_g - r_o) == 1), "a differing intermediate code is not adjacent"
+        # rank 0: the same value with the other sign of zero; rank 1: the
+        # neighbouring code across one rounding boundary
+        assert np.all(np.abs(r_g - r_o) <= 1), "a differing intermediate code is not adjacent"
         s_o = osc[t_i, j_i, c_i // 128].astype(np.float32)
         q_o = (ohf[t_i, j_i, c_i].astype(np.float32) / s_o).astype(np.float64)
         mid = (dec[gc[t_i, j_i, c_i]] + dec[oc[t_i, j_i, c_i]]) / 2
         dist = np.abs(q_o - mid)
         stats["max_mid_dist"] = float(dist.max())
-        assert dist.max() <= mid_tol, (
-            f"a differing code is {dist.max():.3g} scale units from the rounding boundary")
+        lim = mid_tol * np.maximum(np.abs(mid), 1.0)
+        assert np.all(dist <= lim), (
+            f"a differing code is {(dist / lim).max():.3g}x the allowed distance from its rounding boundary")
         wd = h["w_down"].numpy() if hasattr(h["w_down"], "numpy") else h["w_down"]
         sd = h["s_down"].numpy() if hasattr(h["s_down"], "numpy") else h["s_down"]
         for t, j, c in zip(t_i, j_i, c_i):
