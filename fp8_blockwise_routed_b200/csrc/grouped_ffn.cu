@@ -53,10 +53,11 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 128;
-constexpr int STAGES = 4;
+constexpr int A_STAGES = 3;               // activation tiles: L2 hits, short latency
+constexpr int B_STAGES = 5;               // weight tiles: streamed from HBM, long latency
 constexpr int A_TILE = BM * BK;           // 16 KiB
 constexpr int B_HALF = 128 * BK;          // 16 KiB
-constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;
+constexpr int B_TILE = 2 * B_HALF;        // 32 KiB
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 128 + EPI_WARPS * 32;  // 3 warpgroups
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64,512);
@@ -68,19 +69,31 @@ constexpr uint32_t REGS_CTRL = 40;
 constexpr uint32_t REGS_EPI = 232;
 static_assert(128 * REGS_CTRL + 256 * REGS_EPI <= THREADS * 168, "register split exceeds the launch budget");
 static_assert(32 * (REGS_CTRL + 2 * REGS_EPI) <= 16384, "register split exceeds a sub-partition");
-constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_COLS = 512;       // two accumulator buffers of 256 FP32 columns
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr int MAX_E = 1024;
 
-// shared memory map (after the 1024-aligned stage ring)
-constexpr int OFF_BARS = STAGES * STAGE_BYTES;
-constexpr int N_BARS = 2 * STAGES + 4 + 4;  // full, empty, tfull[2], tempty[2], xbar[4]
+// shared memory map (offsets from a 1024-aligned base)
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + A_STAGES * A_TILE;
+constexpr int OFF_BARS = OFF_B + B_STAGES * B_TILE;
+// barriers: fullA, emptyA, fullB, emptyB, tfull[2], tempty[2], xbar[4]
+constexpr int BAR_FULL_A = 0;
+constexpr int BAR_EMPTY_A = BAR_FULL_A + A_STAGES;
+constexpr int BAR_FULL_B = BAR_EMPTY_A + A_STAGES;
+constexpr int BAR_EMPTY_B = BAR_FULL_B + B_STAGES;
+constexpr int BAR_TFULL = BAR_EMPTY_B + B_STAGES;
+constexpr int BAR_TEMPTY = BAR_TFULL + 2;
+constexpr int BAR_XCHG = BAR_TEMPTY + 2;
+constexpr int N_BARS = BAR_XCHG + 4;
 constexpr int OFF_MISC = OFF_BARS + N_BARS * 8;
 constexpr int OFF_AMAX = OFF_MISC + 16;                  // [2 parity][2 half][128 rows] floats
-constexpr int OFF_SEG = OFF_AMAX + 2 * 2 * 128 * 4;      // [MAX_E+1] ints
-constexpr int OFF_IPRE = OFF_SEG + (MAX_E + 1) * 4;      // [MAX_E+1] ints
-constexpr int SMEM_USED = OFF_IPRE + (MAX_E + 1) * 4;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;              // slack for 1024-alignment
+constexpr int OFF_SEG = OFF_AMAX + 2 * 2 * 128 * 4;      // [E+1] ints, then [E+1] ints (item prefix)
+static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && A_TILE % 1024 == 0 && B_TILE % 1024 == 0,
+              "128-byte-swizzled tiles need 1024-byte alignment");
+
+// dynamic shared memory for E experts (plus slack to align the base)
+constexpr int smem_bytes_for(int E) { return OFF_SEG + 2 * (E + 1) * 4 + 1024; }
 
 struct GemmParams {
     int E;
@@ -120,6 +133,9 @@ struct Item {
     int e, nt, mt;
 };
 
+// Work items are ordered expert-major, then n-tile, then m-tile, so that the
+// m-tiles sharing a weight panel are processed at the same time by
+// neighbouring CTAs and share it in L2.
 __device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item)
 {
     Item it;
@@ -133,85 +149,111 @@ __device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int
 
 // ---------------------------------------------------------------- roles
 
+// Weight producer (one lane): the two 128-row weight boxes of every K block
+// into a B_STAGES-deep ring.
 template <int MODE>
-__device__ __forceinline__ void producer_role(const CUtensorMap* tmA, const CUtensorMap* tmB0, const CUtensorMap* tmB1,
-                              const GemmParams& p, const int* seg, const int* ipre, int total_items,
-                              uint32_t sbase, uint32_t bars, volatile int* abort)
+__device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtensorMap* tmB1, const GemmParams& p,
+                                           const int* seg, const int* ipre, int total_items, uint32_t sbase,
+                                           uint32_t bars, volatile int* abort)
 {
-    const uint32_t full0 = bars, empty0 = bars + STAGES * 8;
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        const Item w = decode_item(seg, ipre, p.E, item);
+        const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
+        const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            const int s = it % B_STAGES;
+            if (!mbar_wait_bounded(bars + 8 * (BAR_EMPTY_B + s), ((it / B_STAGES) & 1) ^ 1, abort, WAIT_NS)) {
+                ok = false;
+                break;
+            }
+            const uint32_t fb = bars + 8 * (BAR_FULL_B + s);
+            mbar_arrive_expect_tx(fb, B_TILE);
+            const uint32_t dst = sbase + OFF_B + s * B_TILE;
+            tma_load_3d(dst, tmB0, kb * BK, n0, w.e, fb);
+            tma_load_3d(dst + B_HALF, tmB1, kb * BK, n1, w.e, fb);
+        }
+    }
+    if (!ok) {  // let the copies already issued land before the CTA can exit
+        for (int j = it - B_STAGES > 0 ? it - B_STAGES : 0; j < it; ++j) {
+            volatile int no_abort = 0;
+            mbar_wait_bounded(bars + 8 * (BAR_FULL_B + j % B_STAGES), (j / B_STAGES) & 1, &no_abort, WAIT_NS / 4);
+        }
+    }
+}
+
+// Activation producer (one lane): the 128-row A tile of every K block into
+// an A_STAGES-deep ring.
+__device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmParams& p, const int* seg,
+                                           const int* ipre, int total_items, uint32_t sbase, uint32_t bars,
+                                           volatile int* abort)
+{
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
         const Item w = decode_item(seg, ipre, p.E, item);
         const int row0 = seg[w.e] + w.mt * BM;
-        const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
-        const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1;
-            if (!mbar_wait_bounded(empty0 + 8 * s, ph ^ 1, abort, WAIT_NS)) {
+            const int s = it % A_STAGES;
+            if (!mbar_wait_bounded(bars + 8 * (BAR_EMPTY_A + s), ((it / A_STAGES) & 1) ^ 1, abort, WAIT_NS)) {
                 ok = false;
                 break;
             }
-            const uint32_t fb = full0 + 8 * s;
-            mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            const uint32_t a_dst = sbase + s * STAGE_BYTES;
-            tma_load_2d(a_dst, tmA, kb * BK, row0, fb);
-            tma_load_3d(a_dst + A_TILE, tmB0, kb * BK, n0, w.e, fb);
-            tma_load_3d(a_dst + A_TILE + B_HALF, tmB1, kb * BK, n1, w.e, fb);
+            const uint32_t fb = bars + 8 * (BAR_FULL_A + s);
+            mbar_arrive_expect_tx(fb, A_TILE);
+            tma_load_2d(sbase + OFF_A + s * A_TILE, tmA, kb * BK, row0, fb);
         }
     }
     if (!ok) {
-        // let the copies already issued land before the CTA can exit
-        const int first = it - STAGES > 0 ? it - STAGES : 0;
-        for (int j = first; j < it; ++j) {
+        for (int j = it - A_STAGES > 0 ? it - A_STAGES : 0; j < it; ++j) {
             volatile int no_abort = 0;
-            mbar_wait_bounded(full0 + 8 * (j % STAGES), (j / STAGES) & 1, &no_abort, WAIT_NS / 4);
+            mbar_wait_bounded(bars + 8 * (BAR_FULL_A + j % A_STAGES), (j / A_STAGES) & 1, &no_abort, WAIT_NS / 4);
         }
     }
 }
 
-__device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                         volatile int* abort)
+// MMA issuer (one lane): per K block, four N=256 K=32 MMAs into accumulator
+// buffer it%2 (a fresh accumulation: each 128-deep K block is promoted with
+// its own scales), then commits that free the A and B stages and hand the
+// buffer to the epilogue.
+__device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars,
+                                         uint32_t tmem, volatile int* abort)
 {
-    const int lane = threadIdx.x & 31;
-    const uint32_t full0 = bars, empty0 = bars + STAGES * 8;
-    const uint32_t tfull0 = bars + 2 * STAGES * 8, tempty0 = tfull0 + 16;
     constexpr uint32_t idesc = idesc_e4m3_f32(128, 256);
     int it = 0;
+    int last_commit = -1;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1;
-            const int b = it & 1;
-            const uint32_t bph = (it >> 1) & 1;
-            // every lane waits; the outcome is made warp-uniform so that no
-            // lane is left behind in a warp-synchronous instruction
-            bool ok = mbar_wait_bounded(tempty0 + 8 * b, bph ^ 1, abort, WAIT_NS);
-            ok = ok && mbar_wait_bounded(full0 + 8 * s, ph, abort, WAIT_NS);
-            if (!__all_sync(0xFFFFFFFFu, ok)) goto drain;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t a_addr = sbase + s * STAGE_BYTES;
-                const uint32_t b_addr = a_addr + A_TILE;
+            const int sa = it % A_STAGES, sb = it % B_STAGES, b = it & 1;
+            // no tcgen05 fence after the TMEM wait: the epilogue released the
+            // buffer only after tcgen05.wait::ld, so its reads are complete
+            if (!mbar_spin_bounded(bars + 8 * (BAR_TEMPTY + b), ((it >> 1) & 1) ^ 1, abort, WAIT_NS) ||
+                !mbar_spin_bounded(bars + 8 * (BAR_FULL_B + sb), (it / B_STAGES) & 1, abort, WAIT_NS) ||
+                !mbar_spin_bounded(bars + 8 * (BAR_FULL_A + sa), (it / A_STAGES) & 1, abort, WAIT_NS))
+                goto drain;
+            {
+                const uint32_t a_addr = sbase + OFF_A + sa * A_TILE;
+                const uint32_t b_addr = sbase + OFF_B + sb * B_TILE;
                 const uint32_t d = tmem + b * 256;
 #pragma unroll
                 for (int kk = 0; kk < BK / 32; ++kk)
                     mma_f8(d, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
                            kk > 0 ? 1u : 0u);
-                mma_commit(empty0 + 8 * s);
-                mma_commit(tfull0 + 8 * b);
+                mma_commit(bars + 8 * (BAR_EMPTY_A + sa));
+                mma_commit(bars + 8 * (BAR_EMPTY_B + sb));
+                mma_commit(bars + 8 * (BAR_TFULL + b));
+                last_commit = it;
             }
-            __syncwarp();
         }
     }
     return;
 drain:
     // wait for the MMAs already issued before TMEM is released
-    if (it > 0) {
+    if (last_commit >= 0) {
         volatile int no_abort = 0;
-        const int last = it - 1;
-        mbar_wait_bounded(tfull0 + 8 * (last & 1), (last >> 1) & 1, &no_abort, WAIT_NS / 4);
+        mbar_wait_bounded(bars + 8 * (BAR_TFULL + (last_commit & 1)), (last_commit >> 1) & 1, &no_abort,
+                          WAIT_NS / 4);
     }
 }
 
@@ -224,7 +266,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 4) >> 2;        // column half-slice of each 128-wide half
     const int trow = q * 32 + lane;          // row within the tile
-    const uint32_t tfull0 = bars + 2 * STAGES * 8, tempty0 = tfull0 + 16, xbar0 = tempty0 + 16;
+    const uint32_t tfull0 = bars + 8 * BAR_TFULL, tempty0 = bars + 8 * BAR_TEMPTY, xbar0 = bars + 8 * BAR_XCHG;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     int it = 0;
     int nitem = 0;
@@ -254,8 +296,6 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
         // scales of K block kb+1 are fetched while block kb is promoted
         float sa_n = __ldg(sa_row), w0_n = __ldg(s0), w1_n = has1 ? __ldg(s1) : 0.f;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-            const int b = it & 1;
-            const uint32_t bph = (it >> 1) & 1;
             const float c0 = sa_n * w0_n;
             const float c1 = sa_n * w1_n;
             if (kb + 1 < p.num_kb) {
@@ -263,11 +303,14 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                 w0_n = __ldg(s0 + kb + 1);
                 if (has1) w1_n = __ldg(s1 + kb + 1);
             }
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, bph, abort, WAIT_NS))) return;
-            tc_fence_after();
+            // buffer it%2 holds the partial of this K block: columns [0,128)
+            // -> acc0 (gate / first output block), [128,256) -> acc1; this
+            // thread reads its 64 columns of each half in 32-column loads,
+            // each load overlapping the FMAs of the one before, and releases
+            // the buffer as soon as the last load has landed
+            const int b = it & 1;
+            if (!__all_sync(0xFFFFFFFFu, mbar_spin_bounded(tfull0 + 8 * b, (it >> 1) & 1, abort, WAIT_NS))) return;
             const uint32_t col = lane_base + b * 256 + half * 64;
-            // four 32-column loads; each load after the first overlaps the
-            // FMAs of the one before
             uint32_t ra[32], rb[32];
             tmem_ld32_issue(col, ra);
             tmem_ld_wait(ra);
@@ -283,11 +326,10 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
 #pragma unroll
             for (int i = 0; i < 32; ++i) acc1[i] = fmaf(c1, __uint_as_float(ra[i]), acc1[i]);
             tmem_ld_wait(rb);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(c1, __uint_as_float(rb[i]), acc1[32 + i]);
-            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty0 + 8 * b);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(c1, __uint_as_float(rb[i]), acc1[32 + i]);
         }
 
         if (MODE == 0) {
@@ -300,9 +342,10 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 const float g = acc0[i];
-                // SiLU(g) = g / (1 + exp(-g)), as g times the correctly
-                // rounded reciprocal (within 1.5 ulp of the quotient)
-                const float h = g * __frcp_rn(1.0f + expf(-g)) * acc1[i];
+                // SiLU(g) = g / (1 + exp(-g)) with the hardware exp2 and
+                // divide approximations (a few ulp; the requantisation below
+                // is insensitive to that except within it of a boundary)
+                const float h = __fdividef(g, 1.0f + exp2f(-g * 1.4426950408889634f)) * acc1[i];
                 acc0[i] = h;
                 if (isfinite(h)) amax = fmaxf(amax, fabsf(h));
                 else bad = 1;
@@ -312,7 +355,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             __syncwarp();
             if (lane == 0) mbar_arrive(xbar0 + 8 * q);
             if (!__all_sync(0xFFFFFFFFu,
-                            mbar_wait_bounded(xbar0 + 8 * q, static_cast<uint32_t>(nitem & 1), abort, WAIT_NS)))
+                            mbar_spin_bounded(xbar0 + 8 * q, static_cast<uint32_t>(nitem & 1), abort, WAIT_NS)))
                 return;
             const float other = amax_x[(par * 2 + (half ^ 1)) * 128 + trow];
             const bool nonfinite = bad || isinf(other);
@@ -394,20 +437,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* bad = reinterpret_cast<int*>(smem + OFF_MISC + 8);
     float* amax_x = reinterpret_cast<float*>(smem + OFF_AMAX);
     int* seg = reinterpret_cast<int*>(smem + OFF_SEG);
-    int* ipre = reinterpret_cast<int*>(smem + OFF_IPRE);
+    int* ipre = seg + (p.E + 1);
     const int warp = threadIdx.x >> 5;
     const int E = p.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(bars + 8 * s, 1);                 // full: producer arrive + tx
-            mbar_init(bars + 8 * (STAGES + s), 1);      // empty: MMA commit
+        for (int s = 0; s < A_STAGES; ++s) {
+            mbar_init(bars + 8 * (BAR_FULL_A + s), 1);   // producer arrive + tx
+            mbar_init(bars + 8 * (BAR_EMPTY_A + s), 1);  // MMA commit
+        }
+        for (int s = 0; s < B_STAGES; ++s) {
+            mbar_init(bars + 8 * (BAR_FULL_B + s), 1);
+            mbar_init(bars + 8 * (BAR_EMPTY_B + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(bars + 8 * (2 * STAGES + b), 1);              // tfull: MMA commit
-            mbar_init(bars + 8 * (2 * STAGES + 2 + b), EPI_WARPS);  // tempty: epilogue warps
+            mbar_init(bars + 8 * (BAR_TFULL + b), 1);           // MMA commit
+            mbar_init(bars + 8 * (BAR_TEMPTY + b), EPI_WARPS);  // epilogue warps
         }
-        for (int q = 0; q < 4; ++q) mbar_init(bars + 8 * (2 * STAGES + 4 + q), 2);  // amax exchange
+        for (int q = 0; q < 4; ++q) mbar_init(bars + 8 * (BAR_XCHG + q), 2);  // amax exchange
         *abort = 0;
         *bad = 0;
         fence_barrier_init();
@@ -448,11 +495,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp < 4) {
         setmaxnreg_dec<REGS_CTRL>();
-        if (warp == 0) {
-            if ((threadIdx.x & 31) == 0)
-                producer_role<MODE>(&tmA, &tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
-        } else if (warp == 1) {
-            mma_role(p, total_items, sbase, bars, tmem, abort);
+        if ((threadIdx.x & 31) == 0) {
+            if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
+            else if (warp == 1) mma_role(p, total_items, sbase, bars, tmem, abort);
+            else if (warp == 3) producer_a(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {
         setmaxnreg_inc<REGS_EPI>();
@@ -541,16 +587,17 @@ template <int MODE>
 cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                      int grid, cudaStream_t s)
 {
+    const int smem = smem_bytes_for(MAX_E);
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
         cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
         attr_done[dev] = true;
     }
-    grouped_gemm_kernel<MODE><<<grid, THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
+    grouped_gemm_kernel<MODE><<<grid, THREADS, smem_bytes_for(p.E), s>>>(a, b0, b1, p);
     return cudaGetLastError();
 }
 
@@ -588,7 +635,7 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     if (P == 0) return cudaSuccess;
     DeviceInfo di;
     if (!device_info(&di)) return cudaErrorUnknown;
-    if (di.max_smem_optin < static_cast<size_t>(SMEM_BYTES)) return cudaErrorNotSupported;
+    if (di.max_smem_optin < static_cast<size_t>(smem_bytes_for(MAX_E))) return cudaErrorNotSupported;
     const int H = a.H, I = a.I, E = a.E;
     const int GH = H / 128, GI = (I + 127) / 128, Ip = GI * 128;
 
