@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
         L.moe_route_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_route.restype = i32
         L.moe_route.argtypes = [P, i64, i32, i32, P, P, P, P, P, sz, P]
+        L.moe_route_noalloc.restype = i32
+        L.moe_route_noalloc.argtypes = [P, i64, i32, i32, P, P, P, P, P]
+        L.moe_route_noalloc_error.restype = ctypes.c_char_p
+        L.moe_route_noalloc_error.argtypes = []
         L.moe_quant_act.restype = i32
         L.moe_quant_act.argtypes = [P, i64, i32, P, P, P]
         L.moe_ffn_workspace_bytes.restype = sz
@@ -117,6 +121,17 @@ def moe_route(logits, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws,
     T, E = logits.shape
     _check(lib().moe_route(_p(logits), T, E, top_k, _p(topk_ids), _p(topk_w), _p(expert_offsets),
                            _p(sorted_pairs), _p(ws), ws.numel() * ws.element_size(), _s(stream)), "moe_route")
+
+
+def moe_route_noalloc(logits, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, stream=None):
+    """moe_route for callers that cannot allocate device memory: no workspace;
+    the library's static device scratch is used instead (calls that overlap
+    on the GPU race; see the header)."""
+    T, E = logits.shape
+    code = lib().moe_route_noalloc(_p(logits), T, E, top_k, _p(topk_ids), _p(topk_w), _p(expert_offsets),
+                                   _p(sorted_pairs), _s(stream))
+    if code != 0:
+        raise MoeError(code, "moe_route_noalloc", lib().moe_route_noalloc_error().decode())
 
 
 def moe_quant_act(x, codes, scales, stream=None):

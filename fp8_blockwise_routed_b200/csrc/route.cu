@@ -25,7 +25,10 @@
 // any launch shape and from run to run.
 #include <cfloat>
 #include <climits>
+#include <cstdio>
+#include <mutex>
 
+#include "../../include/fp8moe.h"
 #include "internal.h"
 
 namespace fp8moe {
@@ -241,3 +244,95 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
 }
 
 }  // namespace fp8moe
+
+// ---------------------------------------------------------------------------
+// moe_route_noalloc: moe_route for callers that cannot allocate device
+// memory at all -- not even the small workspace moe_route asks for.  Typical
+// cases: code running inside another runtime's execution hook (an inference
+// engine plugin, a custom op inside a framework that owns and pre-plans every
+// device byte), or latency-critical paths where the implicit device
+// synchronisation of cudaMalloc/cudaFree is not acceptable.  The scratch the
+// router needs lives in one file-scope device array instead, which every GPU
+// that loads this library holds until the process exits.
+namespace {
+
+// Route scratch for one call: block histograms ceil(T/128) x E int32, then
+// per-pair block ranks T*top_k int32 (each region 256-byte aligned).  1 MiB
+// + 4 KiB covers, for example, T = 16384 tokens with E = 1024 experts and
+// top_k = 8.
+constexpr size_t kNoAllocScratchBytes = (size_t(1) << 20) + 4096;
+__device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+// Device address of g_route_scratch, looked up once per device with that
+// device current (in host code the symbol is only a host-side stand-in and
+// must not be passed to a kernel).
+void* scratch_address(int dev, cudaError_t* err)
+{
+    static void* addr[64] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    *err = cudaSuccess;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    if (!addr[dev]) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+thread_local char g_noalloc_error[160] = "";
+
+}  // namespace
+
+extern "C" const char* moe_route_noalloc_error(void) { return g_noalloc_error; }
+
+extern "C" int moe_route_noalloc(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids,
+                                 float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs, void* stream)
+{
+    using namespace fp8moe;
+    g_noalloc_error[0] = 0;
+    if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 0 || top_k > E || top_k > MOE_MAX_TOP_K)
+        return MOE_ERR_INVALID_ARG;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && top_k > 0 && (!logits || !topk_ids || !topk_w || !sorted_pairs)) return MOE_ERR_INVALID_ARG;
+    auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (!al(logits) || !al(topk_ids) || !al(topk_w) || !al(expert_offsets) || !al(sorted_pairs))
+        return MOE_ERR_ALIGNMENT;
+    // the same scratch layout moe_route uses inside its workspace
+    const int64_t nblocks = ceil_div64(T > 0 ? T : 1, kRouteTokensPerBlock);
+    const size_t off_hist = 256;
+    const size_t off_rank = align_up(off_hist + static_cast<size_t>(nblocks) * E * 4, 256);
+    const size_t need = align_up(off_rank + static_cast<size_t>(T > 0 ? T : 1) * (top_k > 0 ? top_k : 1) * 4, 256);
+    if (need > kNoAllocScratchBytes) {
+        std::snprintf(g_noalloc_error, sizeof(g_noalloc_error),
+                      "route scratch for T=%lld E=%d top_k=%d is %zu bytes; the static array holds %zu",
+                      static_cast<long long>(T), E, top_k, need, kNoAllocScratchBytes);
+        return MOE_ERR_WORKSPACE;
+    }
+    DeviceInfo di;
+    if (!device_info(&di)) return MOE_ERR_CUDA;
+    if (di.major != 10 || di.minor != 0) return MOE_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t err;
+    uint8_t* base = static_cast<uint8_t*>(scratch_address(dev, &err));
+    if (!base) {
+        std::snprintf(g_noalloc_error, sizeof(g_noalloc_error), "cudaGetSymbolAddress: %s", cudaGetErrorString(err));
+        return MOE_ERR_CUDA;
+    }
+    // Nothing in the array has to start at zero: every call writes the
+    // histograms and ranks it later reads.
+    err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
+                       reinterpret_cast<int32_t*>(base + off_hist), reinterpret_cast<int32_t*>(base + off_rank),
+                       static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) {
+        std::snprintf(g_noalloc_error, sizeof(g_noalloc_error), "launch: %s", cudaGetErrorString(err));
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}

@@ -136,6 +136,34 @@ MOE_API int moe_route(const float* logits, int64_t T, int E, int top_k,
               void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_noalloc -- moe_route without a workspace argument.  The pages
+ * have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory at all (for example code running inside another
+ * runtime's execution hook, which owns and pre-plans every device byte, or
+ * a latency-critical path that cannot afford the implicit synchronisation of
+ * cudaMalloc).  It allocates nothing; the router's scratch (block histograms
+ * and per-pair ranks) lives in one static device array of 1 MiB + 4 KiB that
+ * every GPU loading the library holds until the process exits.
+ *   - Same arguments, results and limits as moe_route, and additionally the
+ *     scratch of (T, E, top_k) must fit the array: ceil(T/128)*E*4 +
+ *     T*top_k*4 bytes plus alignment (T = 16384, E = 1024, top_k = 8 fits).
+ *     Larger requests return MOE_ERR_WORKSPACE before anything is enqueued;
+ *     moe_route_noalloc_error() then names the sizes.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array: calls whose kernels overlap on the GPU
+ *     (other streams, other host threads) race with each other.  Serialise
+ *     them, e.g. on one stream.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route_noalloc(const float* logits, int64_t T, int E, int top_k,
+                              int32_t* topk_ids, float* topk_w,
+                              int32_t* expert_offsets, int32_t* sorted_pairs, void* stream);
+/* Text describing the last rejection or failure of moe_route_noalloc on this
+ * thread ("" if none). */
+MOE_API const char* moe_route_noalloc_error(void);
+
+/* ---------------------------------------------------------------------------
  * moe_quant_act -- BF16 activations to E4M3 codes with 1x128 group scales.
  *
  * For each token and each group of 128 consecutive columns:
