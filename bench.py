@@ -114,17 +114,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun sets RANK/LOCAL_RANK/WORLD_SIZE).  The
+    process group carries only barriers and the max of one timing scalar:
+    every rank runs its own batch on its own replica of the weights."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
 
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -134,12 +139,44 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(world, v: float) -> float:
+def max_over_ranks(world, v: float, device="cuda") -> float:
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (and weight replica) from its own seed."""
+    return rank
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step_max: float) -> float:
+    """Weak scaling: every rank processes tokens_per_rank per step; the job's
+    step time is the slowest rank's."""
+    return world * tokens_per_rank / (ms_per_step_max / 1e3)
+
+
+def kernel_source_sha256() -> str:
+    import hashlib
+
+    m = hashlib.sha256()
+    for f in ("grouped_ffn.cu", "sm100.cuh"):
+        m.update(open(os.path.join(ROOT, "fp8_blockwise_routed_b200", "csrc", f), "rb").read())
+    return m.hexdigest()
+
+
+def recorded_traffic(key: str):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    record is missing or the kernel source changed since it was taken."""
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(prof):
+        return None
+    rec = json.load(open(prof))
+    if rec.get("kernel_source_sha256") != kernel_source_sha256():
+        return None
+    return rec.get(key)
 
 
 def gateup_alg_bytes(wl, active: int, P: int) -> float:
@@ -155,16 +192,24 @@ def cpu_baseline(wl, d, budget_tokens: int | None = None):
     sample of the same workload, timed on the host.  Returns tokens/s."""
     import oracle
 
-    n = budget_tokens or 24
     g = mi.generator(0, "cpu_baseline", "cpu")
-    toks = torch.randperm(wl.T, generator=g)[:n].sort().values
-    x = d["x"][toks.to(d["x"].device)].cpu()
-    lg = d["logits"][toks.to(d["logits"].device)].cpu()
+    perm = torch.randperm(wl.T, generator=g)
     W = [d[k].cpu() for k in ("w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down")]
+    xs, ls = d["x"].cpu(), d["logits"].cpu()
     oracle.build()
-    t0 = time.perf_counter()
-    oracle.moe_layer(x, lg, wl.k, *W, wl.routed_scaling)
-    dt = time.perf_counter() - t0
+
+    def run(n):
+        toks = perm[:n].sort().values
+        t0 = time.perf_counter()
+        oracle.moe_layer(xs[toks], ls[toks], wl.k, *W, wl.routed_scaling)
+        return time.perf_counter() - t0
+
+    if budget_tokens:
+        n = budget_tokens
+    else:  # size the sample to 10-20 s of oracle work (a 16-token probe underestimates the rate)
+        probe = min(16, wl.T)
+        n = max(probe, min(wl.T, int(20.0 * probe / max(run(probe), 1e-6))))
+    dt = run(n)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n} seeded tokens of the {wl.name} workload (quantise, route, FFN, combine), "
                       f"{dt:.1f} s"}
@@ -180,7 +225,7 @@ def run_reference(args, wl):
     import oracle
 
     d = mi.make_inputs(wl, 0, "cpu")
-    n = 8
+    n = 32  # tokens per step: about a third of a second of oracle work on 16 cores
     W = [d[k] for k in ("w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down")]
     oracle.build()
 
@@ -231,9 +276,9 @@ def main():
 
     import fp8_blockwise_routed_b200 as fm
 
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = dist_setup("nccl")
     dev = torch.device("cuda", torch.cuda.current_device())
-    d = mi.make_inputs(wl, seed=rank, device=dev)
+    d = mi.make_inputs(wl, seed=rank_seed(rank), device=dev)
     layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"],
                          wl.k, wl.routed_scaling, wl.T)
     s = torch.cuda.current_stream()
@@ -291,11 +336,7 @@ def main():
     layer_bytes = mi.algorithmic_bytes(wl, active)
     roof_s = max(flops / (fp8_peak * 1e12), (layer_bytes - wl.T * wl.H * 4 - wl.T * wl.H * 2 - wl.T * wl.E * 4)
                  / (pk["hbm_gbs"] * 1e9))
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        t = json.load(open(prof)).get(f"gemm_gateup/{wl.name}")
-        traffic = t if t else None
+    traffic = recorded_traffic(f"gemm_gateup/{wl.name}")
 
     # end to end through the C ABI with host buffers
     x_h = d["x"].cpu().pin_memory()
@@ -328,7 +369,7 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": world * wl.T / (ms_step / 1e3),
+            "value": whole_job_tokens_per_s(world, wl.T, ms_step),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -349,7 +390,7 @@ def main():
                              "fp8_peak_tflops": fp8_peak, "roofline_ms": roof_s * 1e3,
                              "frac_roofline": roof_s / gemm_s},
             "stages_ms": stage_ms,
-            "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_tokens_per_s(world, wl.T, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                     "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms},
             "gpu_launches": 8 * args.steps,

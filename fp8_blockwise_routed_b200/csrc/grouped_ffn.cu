@@ -286,6 +286,14 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
         const float* s0 = p.b_s0 + (static_cast<int64_t>(w.e) * p.b_nblocks + nb0) * p.num_kb;
         const float* s1 = p.b_s1 + (static_cast<int64_t>(w.e) * p.b_nblocks + (nb1 < p.b_nblocks ? nb1 : nb0)) * p.num_kb;
         const bool has1 = nb1 < p.b_nblocks;
+        // down: the row's pair index and routing weight, fetched before the
+        // K loop so that the tail does not wait on them
+        int pair = -1;
+        float wt = 0.f;
+        if (MODE == 1 && valid) {
+            pair = __ldg(p.sorted_pairs + r);
+            if (pair >= 0 && pair < p.P) wt = __ldg(p.topk_w + pair);
+        }
 
         float acc0[64], acc1[64];
 #pragma unroll
@@ -395,11 +403,9 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             }
         } else {
             if (valid) {
-                const int pair = __ldg(p.sorted_pairs + r);
                 if (pair < 0 || pair >= p.P) {
                     atomicOr(p.status, kDevBadPair);
                 } else {
-                    const float wt = __ldg(p.topk_w + pair);
                     float* dst = p.y + static_cast<int64_t>(pair) * p.H;
                     const int c0 = w.nt * 256 + half * 64;
                     const int c1 = c0 + 128;

@@ -10,7 +10,7 @@
 // pass routes its experts in one call", "Exactness").
 //
 // Three launches, no host synchronisation, no atomics on the ordering path:
-//   1. route_topk: one warp per token (16 tokens per warp, 8 warps per
+//   1. route_topk: one warp per token (4 tokens per warp, 32 warps per
 //      block).  Logits of a token sit in registers (ceil(E/32) per lane);
 //      k rounds of a warp arg-max (value desc, id asc; NaN and -Inf are
 //      never selected).  Slot weights: expf(l_j - l_0) / sum (FP32).  The
@@ -34,8 +34,8 @@
 namespace fp8moe {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kTokPerWarp = kRouteTokensPerBlock / kWarps;  // 16
+constexpr int kWarps = 32;
+constexpr int kTokPerWarp = kRouteTokensPerBlock / kWarps;  // 4
 
 template <int VPL>
 __global__ void __launch_bounds__(kWarps * 32) route_topk_kernel(const float* __restrict__ logits, int64_t T, int E,
@@ -146,11 +146,17 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ 
     const int lane = e & 31, warp = e >> 5;
     int run = 0;
     if (e < E) {
-        for (int b = 0; b < nblocks; ++b) {
-            const int64_t i = static_cast<int64_t>(b) * E + e;
-            const int c = block_hist[i];
-            block_hist[i] = run;
-            run += c;
+        // batches of independent loads, then their running prefix
+        for (int b0 = 0; b0 < nblocks; b0 += 16) {
+            int c[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                c[j] = (b0 + j < nblocks) ? block_hist[static_cast<int64_t>(b0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (b0 + j < nblocks) block_hist[static_cast<int64_t>(b0 + j) * E + e] = run;
+                run += c[j];
+            }
         }
     }
     int incl = run;

@@ -73,6 +73,9 @@ WORKLOADS = {
     "glm": Workload("glm", 4096, 5120, 256, 8, 1536, 1.0, "normal_outliers", "zipf"),
     "non128": Workload("non128", 2048, 5120, 160, 8, 192, 1.0, "normal", "normal_masked"),
     "long": Workload("long", 16384, 6144, 256, 8, 2048, 1.0, "student_t3", "zipf"),
+    # GLM widths with 64 experts (1.5 GB of weights): the case detailed
+    # profiler captures run on (larger than L2, a few GB on the device)
+    "glm64": Workload("glm64", 2048, 5120, 64, 8, 1536, 1.0, "normal_outliers", "zipf"),
 }
 
 
