@@ -97,6 +97,7 @@ constexpr int smem_bytes_for(int E) { return OFF_SEG + 2 * (E + 1) * 4 + 1024; }
 
 struct GemmParams {
     int E;
+    int rev;               // walk experts last to first (their activation rows were gathered last)
     int num_kb;            // K blocks of 128
     int n_tiles;           // output tiles per expert along N
     int64_t P;             // rows of the pair buffers (T * top_k)
@@ -114,6 +115,7 @@ struct GemmParams {
     const int32_t* sorted_pairs;
     const float* topk_w;
     float* y;              // [P, H]
+    int y_v8;              // y is 32-byte aligned: 32-byte stores
     int H;
     int* status;
 };
@@ -136,11 +138,12 @@ struct Item {
 // Work items are ordered expert-major, then n-tile, then m-tile, so that the
 // m-tiles sharing a weight panel are processed at the same time by
 // neighbouring CTAs and share it in L2.
-__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item)
+__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item, int rev)
 {
     Item it;
-    it.e = find_expert(ipre, E, item);
-    const int local = item - ipre[it.e];
+    const int o = find_expert(ipre, E, item);  // position of the expert in the walk order
+    it.e = rev ? E - 1 - o : o;
+    const int local = item - ipre[o];
     const int mts = (seg[it.e + 1] - seg[it.e] + BM - 1) / BM;
     it.nt = local / mts;
     it.mt = local - it.nt * mts;
@@ -159,7 +162,7 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
         const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
         const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
@@ -192,7 +195,7 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
         const int row0 = seg[w.e] + w.mt * BM;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             const int s = it % A_STAGES;
@@ -271,7 +274,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
     int it = 0;
     int nitem = 0;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++nitem) {
-        const Item w = decode_item(seg, ipre, p.E, item);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
         const int r = seg[w.e] + w.mt * BM + trow;
         const bool valid = r < seg[w.e + 1];
         const int64_t ra = r < p.P ? r : p.P - 1;
@@ -409,19 +412,37 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                     float* dst = p.y + static_cast<int64_t>(pair) * p.H;
                     const int c0 = w.nt * 256 + half * 64;
                     const int c1 = c0 + 128;
-                    if (c0 < p.H) {
+                    // 32-byte stores (whole sectors) when y allows, else 16-byte
+                    if (p.y_v8) {
+                        if (c0 < p.H) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            reinterpret_cast<float4*>(dst + c0)[c] =
-                                make_float4(wt * acc0[4 * c], wt * acc0[4 * c + 1], wt * acc0[4 * c + 2],
-                                            wt * acc0[4 * c + 3]);
-                    }
-                    if (c1 < p.H) {
+                            for (int c = 0; c < 8; ++c)
+                                st_global_v8(dst + c0 + 8 * c, wt * acc0[8 * c], wt * acc0[8 * c + 1],
+                                             wt * acc0[8 * c + 2], wt * acc0[8 * c + 3], wt * acc0[8 * c + 4],
+                                             wt * acc0[8 * c + 5], wt * acc0[8 * c + 6], wt * acc0[8 * c + 7]);
+                        }
+                        if (c1 < p.H) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            reinterpret_cast<float4*>(dst + c1)[c] =
-                                make_float4(wt * acc1[4 * c], wt * acc1[4 * c + 1], wt * acc1[4 * c + 2],
-                                            wt * acc1[4 * c + 3]);
+                            for (int c = 0; c < 8; ++c)
+                                st_global_v8(dst + c1 + 8 * c, wt * acc1[8 * c], wt * acc1[8 * c + 1],
+                                             wt * acc1[8 * c + 2], wt * acc1[8 * c + 3], wt * acc1[8 * c + 4],
+                                             wt * acc1[8 * c + 5], wt * acc1[8 * c + 6], wt * acc1[8 * c + 7]);
+                        }
+                    } else {
+                        if (c0 < p.H) {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c)
+                                reinterpret_cast<float4*>(dst + c0)[c] =
+                                    make_float4(wt * acc0[4 * c], wt * acc0[4 * c + 1], wt * acc0[4 * c + 2],
+                                                wt * acc0[4 * c + 3]);
+                        }
+                        if (c1 < p.H) {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c)
+                                reinterpret_cast<float4*>(dst + c1)[c] =
+                                    make_float4(wt * acc1[4 * c], wt * acc1[4 * c + 1], wt * acc1[4 * c + 2],
+                                                wt * acc1[4 * c + 3]);
+                        }
                     }
                 }
             }
@@ -481,12 +502,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         int okv = (seg[0] == 0);
         int acc = 0;
         ipre[0] = 0;
-        for (int e = 0; e < E; ++e) {
+        for (int o = 0; o < E; ++o) {
+            const int e = p.rev ? E - 1 - o : o;  // experts are walked in this order
             const int c = seg[e + 1] - seg[e];
             if (c < 0 || seg[e + 1] > p.P) okv = 0;
             const int mts = c > 0 ? (c + BM - 1) / BM : 0;
             acc += mts * p.n_tiles;
-            ipre[e + 1] = acc;
+            ipre[o + 1] = acc;
         }
         if (!okv) {
             *bad = 1;
@@ -684,6 +706,7 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     g.P = P;
     g.offsets = a.expert_offsets;
     g.a_scales = a.sa_sorted;
+    g.rev = 1;
     g.b_s0 = a.s_gate;
     g.b_s1 = a.s_up;
     g.b_nblocks = GI;
@@ -708,6 +731,8 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     d.b_s0 = a.s_down;
     d.b_s1 = a.s_down;
     d.b_nblocks = GH;
+    d.rev = 0;
+    d.y_v8 = (reinterpret_cast<uintptr_t>(a.y) & 31u) == 0;
     if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
     if ((err = run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;
     return stage_mark(a, 3, s);
