@@ -28,9 +28,16 @@
 // Warp roles (384 threads, one CTA per SM, grid = #SMs, static round-robin
 // over work items ordered expert-major, then n-tile, then m-tile so that the
 // m-tiles sharing a weight panel run at the same time and share it in L2):
-//   warp 0      TMA producer (one lane): A tile 128x128 B, B tile 2x128x128 B
-//               per stage, 4 stages, mbarrier complete_tx
-//   warp 1      TMEM allocator and MMA issuer (one lane); warps 2-3 idle
+//   warp 0      weight TMA producer (one lane): 2x128x128 B per stage,
+//               B_STAGES deep, mbarrier complete_tx
+//   warp 3      activation TMA producer (one lane): 128x128 B per stage,
+//               A_STAGES deep
+//   warps 1, 2  MMA issuers (one lane each; warp 1 also allocates TMEM):
+//               warp 1 issues the even K blocks, warp 2 the odd ones.  A
+//               thread that issues tcgen05.mma is held while the tensor pipe
+//               works through it, so with one issuer the waits for the next
+//               block's operands and buffer could not overlap the MMAs of
+//               the current one; with two, each waits while the other's run.
 //   warps 4..11 promotion + epilogue; warp w reads TMEM lanes 32*(w%4) (its
 //               rows); warps 4..7 own columns [0,64) of each 128-half, warps
 //               8..11 columns [64,128)
@@ -216,18 +223,21 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
     }
 }
 
-// MMA issuer (one lane): per K block, four N=256 K=32 MMAs into accumulator
-// buffer it%2 (a fresh accumulation: each 128-deep K block is promoted with
-// its own scales), then commits that free the A and B stages and hand the
-// buffer to the epilogue.
+// MMA issuer (one lane; two issuers split the K blocks by it%2 == parity, so
+// issuer `parity` always fills accumulator buffer `parity`): per K block,
+// four N=256 K=32 MMAs into the buffer (a fresh accumulation: each 128-deep K
+// block is promoted with its own scales), then commits that free the A and B
+// stages and hand the buffer to the epilogue.  A commit tracks the MMAs of
+// the issuing thread only, which are exactly the ones it hands over.
 __device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars,
-                                         uint32_t tmem, volatile int* abort)
+                                         uint32_t tmem, volatile int* abort, int parity)
 {
     constexpr uint32_t idesc = idesc_e4m3_f32(128, 256);
     int it = 0;
     int last_commit = -1;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            if ((it & 1) != parity) continue;  // the other issuer's K block
             const int sa = it % A_STAGES, sb = it % B_STAGES, b = it & 1;
             // no tcgen05 fence after the TMEM wait: the epilogue released the
             // buffer only after tcgen05.wait::ld, so its reads are complete
@@ -525,7 +535,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         setmaxnreg_dec<REGS_CTRL>();
         if ((threadIdx.x & 31) == 0) {
             if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
-            else if (warp == 1) mma_role(p, total_items, sbase, bars, tmem, abort);
+            else if (warp == 1 || warp == 2) mma_role(p, total_items, sbase, bars, tmem, abort, warp - 1);
             else if (warp == 3) producer_a(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {
