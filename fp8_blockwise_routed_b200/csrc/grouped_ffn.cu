@@ -330,7 +330,10 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             // each load overlapping the FMAs of the one before, and releases
             // the buffer as soon as the last load has landed
             const int b = it & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_spin_bounded(tfull0 + 8 * b, (it >> 1) & 1, abort, WAIT_NS))) return;
+            // a suspending wait: the epilogue warps share their sub-partitions
+            // with the producer and issuer lanes, which a polling loop would
+            // take issue slots from
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, (it >> 1) & 1, abort, WAIT_NS))) return;
             const uint32_t col = lane_base + b * 256 + half * 64;
             uint32_t ra[32], rb[32];
             tmem_ld32_issue(col, ra);
@@ -358,28 +361,31 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             // this row's 128 intermediate columns [nt*128, nt*128+128), half of
             // which this thread holds; the other half comes through shared
             // memory from the partner warp of the same lane quarter.
+            // amax is NaN-propagating, so it is finite exactly when every h
+            // of this half-row is
             float amax = 0.f;
-            int bad = 0;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 const float g = acc0[i];
-                // SiLU(g) = g / (1 + exp(-g)) with the hardware exp2 and
-                // divide approximations (a few ulp; the requantisation below
-                // is insensitive to that except within it of a boundary)
-                const float h = __fdividef(g, 1.0f + exp2f(-g * 1.4426950408889634f)) * acc1[i];
+                // SiLU(g) = g / (1 + e^-g), e^-g = 2^(-g log2 e), with the
+                // hardware exp2 and reciprocal approximations (a few ulp; the
+                // requantisation below is insensitive to that except within
+                // it of a rounding boundary).  e^-g overflows to +inf for
+                // g < -88.7, where the reciprocal gives 0 and h = -0 * u.
+                const float e = ex2_approx_ftz(-g * 1.4426950408889634f);
+                const float h = (g * rcp_approx_ftz(1.0f + e)) * acc1[i];
                 acc0[i] = h;
-                if (isfinite(h)) amax = fmaxf(amax, fabsf(h));
-                else bad = 1;
+                amax = fmax_nan(amax, fabsf(h));
             }
             const int par = nitem & 1;
-            amax_x[(par * 2 + half) * 128 + trow] = bad ? INFINITY : amax;
+            amax_x[(par * 2 + half) * 128 + trow] = amax;
             __syncwarp();
             if (lane == 0) mbar_arrive(xbar0 + 8 * q);
             if (!__all_sync(0xFFFFFFFFu,
                             mbar_spin_bounded(xbar0 + 8 * q, static_cast<uint32_t>(nitem & 1), abort, WAIT_NS)))
                 return;
             const float other = amax_x[(par * 2 + (half ^ 1)) * 128 + trow];
-            const bool nonfinite = bad || isinf(other);
+            const bool nonfinite = !isfinite(amax) || !isfinite(other);
             float s = __fdiv_rn(fmaxf(amax, other), 448.0f);
             if (s == 0.f) s = 1.f;
             if (valid) {
@@ -396,18 +402,20 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                     // E4M3 rounding boundary).  Scales whose reciprocal
                     // overflows use the divide.
                     const float inv = __frcp_rn(s);
-                    const bool use_div = !isfinite(inv);
+                    if (!isfinite(inv)) {  // rare: divide each value
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) acc0[i] = __fdiv_rn(acc0[i], s);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) acc0[i] *= inv;
+                    }
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t wv[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const int i = c * 16 + j * 4;
-                            float q[4];
-#pragma unroll
-                            for (int m = 0; m < 4; ++m)
-                                q[m] = use_div ? __fdiv_rn(acc0[i + m], s) : acc0[i + m] * inv;
-                            wv[j] = e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16);
+                            wv[j] = e4m3x2(acc0[i], acc0[i + 1]) | (e4m3x2(acc0[i + 2], acc0[i + 3]) << 16);
                         }
                         reinterpret_cast<uint4*>(dst)[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                     }

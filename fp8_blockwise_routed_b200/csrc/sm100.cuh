@@ -311,6 +311,28 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
            | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
 }
 
+// Hardware approximations (MUFU): 2^x and 1/x, subnormal inputs and
+// results flushed to zero.
+__device__ __forceinline__ float ex2_approx_ftz(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx_ftz(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// max that returns NaN if either operand is NaN.
+__device__ __forceinline__ float fmax_nan(float a, float b)
+{
+    float y;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+    return y;
+}
+
 // E4M3 pair encode, round to nearest even, saturating (NaN -> 0x7F).
 // Returns lo in bits 0..7 and hi in bits 8..15.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
