@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference] [--workload glm]
 
-One step = one whole layer call (moe_quant_act, moe_route, moe_grouped_ffn,
+One step = one whole layer call (moe_route_quant, moe_grouped_ffn,
 moe_combine) over one batch of T tokens, inputs resident in HBM.  Workload:
 the GLM-class layer (T=4096, H=5120, 256 experts, top-8, I=1536, 0.1 %
 outlier tokens x100, Zipf(1.1) routing), the configuration the throughput
@@ -18,7 +18,7 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
   cpu_baseline  the oracle (plain C, FP64) timed on a bounded token sample
                 on this host's cores;
   e2e           the same metric with host buffers: pinned H2D of x and
-                logits, the four calls, D2H of the FP32 output, per step;
+                logits, the three calls, D2H of the FP32 output, per step;
   stages        per-launch-group milliseconds from CUDA events;
   clocks        nvidia-smi samples taken during the timed region.
 """
@@ -42,6 +42,9 @@ import torch  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 
 METRIC = "routed-MoE prefill tokens/s per layer; grouped-GEMM % of B200 FP8 peak"
+# kernels of libfp8moe per layer call: route_topk (+ quantiser), route_rank,
+# route_scatter, gather_rows, grouped_gemm<0>, grouped_gemm<1>, combine
+LAUNCHES_PER_LAYER = 7
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -318,9 +321,12 @@ def main():
     ms_total = max_over_ranks(world, t0.elapsed_time(t1))
     ms_step = ms_total / args.steps
     status = layer.device_status()
-    names = ["quant_act", "route", "gather", "gemm_gateup", "gemm_down", "combine"]
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
-                for j, n in enumerate(names)}
+    # forward's events: 0 start, (1 = 0 when fused), 2 gather, 3 gate/up,
+    # 4 down, 5 combine, 6 end
+    spans = {"route_quant": (0, 2), "gather": (2, 3), "gemm_gateup": (3, 4), "gemm_down": (4, 5),
+             "combine": (5, 6)}
+    stage_ms = {n: statistics.mean(evs[i][a].elapsed_time(evs[i][b]) for i in range(args.steps))
+                for n, (a, b) in spans.items()}
 
     # roofline of the dominant kernel
     pk = peaks()
@@ -393,7 +399,7 @@ def main():
             "e2e": {"value": whole_job_tokens_per_s(world, wl.T, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                     "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms},
-            "gpu_launches": 8 * args.steps,
+            "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
             "device_status": status,
             "active_experts": active,
             "pairs": P,

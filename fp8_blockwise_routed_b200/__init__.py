@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc_error.argtypes = []
         L.moe_quant_act.restype = i32
         L.moe_quant_act.argtypes = [P, i64, i32, P, P, P]
+        L.moe_route_quant.restype = i32
+        L.moe_route_quant.argtypes = [P, P, i64, i32, i32, i32, P, P, P, P, P, P, P, sz, P]
         L.moe_ffn_workspace_bytes.restype = sz
         L.moe_ffn_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
         L.moe_grouped_ffn.restype = i32
@@ -139,6 +141,18 @@ def moe_quant_act(x, codes, scales, stream=None):
     _check(lib().moe_quant_act(_p(x), T, H, _p(codes), _p(scales), _s(stream)), "moe_quant_act")
 
 
+def moe_route_quant(logits, x, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, codes, scales, ws,
+                    stream=None):
+    """moe_route and moe_quant_act in one call (the quantiser rides in the
+    router's first launch); same results as the two calls."""
+    T, E = logits.shape
+    H = x.shape[1]
+    assert x.shape[0] == T
+    _check(lib().moe_route_quant(_p(logits), _p(x), T, H, E, top_k, _p(topk_ids), _p(topk_w), _p(expert_offsets),
+                                 _p(sorted_pairs), _p(codes), _p(scales), _p(ws), ws.numel() * ws.element_size(),
+                                 _s(stream)), "moe_route_quant")
+
+
 def moe_grouped_ffn(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs,
                     w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None, stage_events=None):
     """stage_events: None or 4 torch.cuda.Event objects (already recorded
@@ -194,8 +208,9 @@ def moe_ffn_intermediate(ws, T: int, H: int, I: int, top_k: int):
 class RoutedMoE:
     """One routed-expert layer: resident FP8 weights and their block scales,
     plus output and workspace buffers sized for up to `max_tokens` rows.
-    ``forward`` enqueues moe_quant_act, moe_route, moe_grouped_ffn and
-    moe_combine on the current stream and returns the FP32 output rows."""
+    ``forward`` enqueues moe_route_quant (or, with fused=False, moe_quant_act
+    and moe_route), moe_grouped_ffn and moe_combine on the current stream
+    and returns the FP32 output rows."""
 
     def __init__(self, w_gate, s_gate, w_up, s_up, w_down, s_down, top_k: int, routed_scaling: float,
                  max_tokens: int):
@@ -220,9 +235,10 @@ class RoutedMoE:
         self.ws_comb = torch.empty((moe_combine_workspace_bytes(),), dtype=u8, device=dev)
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, out_bf16: torch.Tensor | None = None,
-                stream=None, stage_events=None) -> torch.Tensor:
+                stream=None, stage_events=None, fused: bool = True) -> torch.Tensor:
         """stage_events: None, or 7 recorded torch.cuda.Events marking the
-        start of quantise, route, gather, gate/up, down, combine and the end."""
+        start of quantise, route, gather, gate/up, down, combine and the end
+        (fused: the first two both mark the start of moe_route_quant)."""
         T = x.shape[0]
         assert T <= self.max_tokens and x.shape[1] == self.H and logits.shape == (T, self.E)
         codes, scales = self.codes[:T], self.scales[:T]
@@ -232,10 +248,15 @@ class RoutedMoE:
         s = torch.cuda.current_stream() if stream is None else stream
         if ev is not None:
             ev[0].record(s)
-        moe_quant_act(x, codes, scales, stream)
-        if ev is not None:
-            ev[1].record(s)
-        moe_route(logits, self.k, ids, tw, self.offsets, srt, self.ws_route, stream)
+        if fused:
+            if ev is not None:
+                ev[1].record(s)
+            moe_route_quant(logits, x, self.k, ids, tw, self.offsets, srt, codes, scales, self.ws_route, stream)
+        else:
+            moe_quant_act(x, codes, scales, stream)
+            if ev is not None:
+                ev[1].record(s)
+            moe_route(logits, self.k, ids, tw, self.offsets, srt, self.ws_route, stream)
         moe_grouped_ffn(codes, scales, ids, tw, self.offsets, srt, *self.w, y, self.ws_ffn, stream,
                         stage_events=None if ev is None else ev[2:6])
         moe_combine(y, ids, self.E, self.rs, out, out_bf16, self.ws_comb, stream)

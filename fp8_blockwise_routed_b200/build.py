@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfp8moe.so")
 SOURCES = ["api.cu", "route.cu", "quant_act.cu", "combine.cu", "grouped_ffn.cu"]
-HEADERS = ["internal.h", "sm100.cuh"]
+HEADERS = ["internal.h", "sm100.cuh", "quant_body.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -84,10 +84,14 @@ int clear_status(void* ws, cudaStream_t s)
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "status clear");
 }
 
-size_t route_layout(int64_t T, int E, int k, size_t* off_hist, size_t* off_rank)
+// Route workspace: status word, arrival counter (256 bytes), block histograms
+// [ceil(T/128), E] i32, pair ranks [T*k] i32.
+size_t route_layout(int64_t T, int E, int k, size_t* off_arr, size_t* off_hist, size_t* off_rank)
 {
     const int64_t nblocks = ceil_div64(T > 0 ? T : 1, kRouteTokensPerBlock);
     size_t o = kStatusBytes;
+    *off_arr = o;
+    o += 256;
     *off_hist = o;
     o = align_up(o + static_cast<size_t>(nblocks) * (E > 0 ? E : 1) * 4, 256);
     *off_rank = o;
@@ -120,12 +124,15 @@ const char* moe_last_error(void) { return g_last_error; }
 size_t moe_route_workspace_bytes(int64_t T, int E, int top_k)
 {
     if (T < 0 || E < 1 || top_k < 0) return 0;
-    size_t a, b;
-    return route_layout(T, E, top_k, &a, &b);
+    size_t a, b, c;
+    return route_layout(T, E, top_k, &a, &b, &c);
 }
 
-int moe_route(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
-              int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream)
+namespace {
+
+int route_common(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
+                 int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream,
+                 const fp8moe::QuantArgs* quant, const char* what)
 {
     if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 0 || top_k > E || top_k > MOE_MAX_TOP_K)
         return MOE_ERR_INVALID_ARG;
@@ -135,16 +142,37 @@ int moe_route(const float* logits, int64_t T, int E, int top_k, int32_t* topk_id
     if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) ||
         !aligned16(sorted_pairs) || !aligned16(ws))
         return MOE_ERR_ALIGNMENT;
-    size_t off_hist, off_rank;
-    if (ws_bytes < route_layout(T, E, top_k, &off_hist, &off_rank)) return MOE_ERR_WORKSPACE;
+    size_t off_arr, off_hist, off_rank;
+    if (ws_bytes < route_layout(T, E, top_k, &off_arr, &off_hist, &off_rank)) return MOE_ERR_WORKSPACE;
     if (int r = check_device()) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (int r = clear_status(ws, s)) return r;
     uint8_t* w8 = static_cast<uint8_t*>(ws);
     cudaError_t err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
                                    reinterpret_cast<int32_t*>(w8 + off_hist), reinterpret_cast<int32_t*>(w8 + off_rank),
-                                   s);
-    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route");
+                                   reinterpret_cast<int*>(w8 + off_arr), quant, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, what);
+}
+
+}  // namespace
+
+int moe_route(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
+              int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream)
+{
+    return route_common(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, ws_bytes, stream,
+                        nullptr, "moe_route");
+}
+
+int moe_route_quant(const float* logits, const uint16_t* x, int64_t T, int H, int E, int top_k, int32_t* topk_ids,
+                    float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs, uint8_t* codes, float* scales,
+                    void* ws, size_t ws_bytes, void* stream)
+{
+    if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !codes || !scales)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_ALIGNMENT;
+    const fp8moe::QuantArgs q{x, T, H, codes, scales};
+    return route_common(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, ws_bytes, stream,
+                        &q, "moe_route_quant");
 }
 
 int moe_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* scales, void* stream)

@@ -14,7 +14,8 @@ constexpr int kDevBadPair = 0x2;
 constexpr int kDevBadOffsets = 0x4;
 constexpr int kDevWaitTimeout = 0x8;
 
-// Route kernels: tokens per routing block (8 warps x 16 tokens).
+// Route kernels: tokens per ranking block (the unit of the per-block expert
+// histograms the stable permutation is built from).
 constexpr int kRouteTokensPerBlock = 128;
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -31,9 +32,20 @@ bool device_info(DeviceInfo* out);
 cudaError_t launch_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* scales, cudaStream_t s);
 cudaError_t launch_encode(const float* in, int64_t n, uint8_t* out, cudaStream_t s);
 
+// Activation quantiser work carried by the route's top-k launch.
+struct QuantArgs {
+    const uint16_t* x;  // [T, H] BF16
+    int64_t T;
+    int H;
+    uint8_t* codes;     // [T, H]
+    float* scales;      // [T, H/128]
+};
+
+// block_hist: [ceil(T/128), E] i32; local_rank: [T*k] i32; arrivals: one int
+// (reset by the first launch, counted by the second).  quant may be null.
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w,
                          int32_t* offsets, int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank,
-                         cudaStream_t s);
+                         int* arrivals, const QuantArgs* quant, cudaStream_t s);
 
 cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
                            float* out, uint16_t* out_bf16, int* status, cudaStream_t s);

@@ -10,15 +10,19 @@
 // pass routes its experts in one call", "Exactness").
 //
 // Three launches, no host synchronisation, no atomics on the ordering path:
-//   1. route_topk: one warp per token (4 tokens per warp, 32 warps per
-//      block).  Logits of a token sit in registers (ceil(E/32) per lane);
-//      k rounds of a warp arg-max (value desc, id asc; NaN and -Inf are
-//      never selected).  Slot weights: expf(l_j - l_0) / sum (FP32).  The
-//      same kernel ranks each pair among the block's earlier pairs of the
-//      same expert (per-warp counters in shared memory, tokens in order), and
-//      writes the block's per-expert counts.
-//   2. route_scan: one block; per expert, exclusive prefix of the block
-//      counts in block order, then an exclusive scan over experts.
+//   1. route_topk: one warp per token, 8 tokens per block, so the whole GPU
+//      takes part.  A token's logits sit in registers (ceil(E/32) per
+//      lane); k rounds of a warp arg-max (value desc, id asc; NaN and -Inf
+//      are never selected).  Slot weights: expf(l_j - l_0) / sum (FP32).
+//      The same launch can carry the activation quantiser in its trailing
+//      blocks (moe_route_quant), which needs no routing result.
+//   2. route_rank: one block per 128 tokens.  A pair's rank among the
+//      block's earlier pairs of the same expert comes from a warp match
+//      (lanes in order) plus per-warp counts in shared memory (warps in
+//      order); the block writes its per-expert counts.  The last block to
+//      finish (an arrival counter) scans the counts: per expert, exclusive
+//      prefix over blocks in block order, then an exclusive scan over
+//      experts -> expert_offsets.
 //   3. route_scatter: pair p goes to offsets[e] + base[block(p)][e] +
 //      rank_in_block(p); positions past offsets[E] get -1.
 // Every integer output is a pure function of the ids, so it is the same for
@@ -30,128 +34,157 @@
 
 #include "../../include/fp8moe.h"
 #include "internal.h"
+#include "quant_body.cuh"
 
 namespace fp8moe {
 namespace {
 
-constexpr int kWarps = 32;
-constexpr int kTokPerWarp = kRouteTokensPerBlock / kWarps;  // 4
+constexpr int kTopkWarps = 8;     // tokens per top-k block
+constexpr int kRankThreads = 1024;
 
+// Top-k of one token by one warp; writes ids[t*k + j], w[t*k + j].
 template <int VPL>
-__global__ void __launch_bounds__(kWarps * 32) route_topk_kernel(const float* __restrict__ logits, int64_t T, int E,
-                                                                 int k, int32_t* __restrict__ ids,
-                                                                 float* __restrict__ w,
-                                                                 int32_t* __restrict__ block_hist,
-                                                                 int32_t* __restrict__ local_rank)
+__device__ __forceinline__ void topk_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ ids,
+                                           float* __restrict__ w, int lane)
 {
-    extern __shared__ int32_t sm[];
-    int32_t* warp_cnt = sm;                                     // [kWarps][E]
-    int32_t* s_rank = sm + kWarps * E;                          // [128][k]
-    int32_t* s_id = s_rank + kRouteTokensPerBlock * k;          // [128][k]
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) warp_cnt[i] = 0;
-    for (int i = threadIdx.x; i < kRouteTokensPerBlock * k; i += blockDim.x) s_id[i] = -1;
-    __syncthreads();
-
-    const int64_t blk_tok0 = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock;
-    for (int tt = 0; tt < kTokPerWarp; ++tt) {
-        const int tl = warp * kTokPerWarp + tt;  // token index within the block
-        const int64_t t = blk_tok0 + tl;
-        if (t >= T) break;
-        const float* row = logits + t * E;
-        float v[VPL];
+    float v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+    }
+    uint32_t taken = 0;
+    int my_id = -1;
+    float my_val = 0.0f, top = 0.0f;
+    int nsel = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = INT_MAX;
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
             const int e = lane + 32 * i;
-            v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
-        }
-        uint32_t taken = 0;
-        int my_id = -1;
-        float my_val = 0.0f, top = 0.0f;
-        int nsel = 0;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = INT_MAX;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int e = lane + 32 * i;
-                const bool sel = (e < E) && !((taken >> i) & 1u) && !isnan(v[i]) && v[i] != -INFINITY;
-                if (sel && (be == INT_MAX || v[i] > bv)) {  // ascending e: strict '>' keeps the lower id
-                    bv = v[i];
-                    be = e;
-                }
+            const bool sel = (e < E) && !((taken >> i) & 1u) && !isnan(v[i]) && v[i] != -INFINITY;
+            if (sel && (be == INT_MAX || v[i] > bv)) {  // ascending e: strict '>' keeps the lower id
+                bv = v[i];
+                be = e;
             }
+        }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-                const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-                if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-                    bv = ov;
-                    be = oe;
-                }
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+            if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
             }
-            if (be == INT_MAX) break;  // nothing selectable is left
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == j) {
-                my_id = be;
-                my_val = bv;
-            }
-            if (j == 0) top = bv;
-            ++nsel;
         }
-        const float ex = (lane < nsel) ? expf(my_val - top) : 0.0f;
-        float sum = ex;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-        if (lane < k) {
-            ids[t * k + lane] = (lane < nsel) ? my_id : -1;
-            w[t * k + lane] = (lane < nsel) ? __fdiv_rn(ex, sum) : 0.0f;
+        if (be == INT_MAX) break;  // nothing selectable is left
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) {
+            my_id = be;
+            my_val = bv;
         }
-        // stable rank among this warp's earlier pairs of the same expert; a
-        // token's selected experts are distinct, so lanes never collide
-        if (lane < nsel) {
-            const int c = warp_cnt[warp * E + my_id];
-            s_rank[tl * k + lane] = c;
-            s_id[tl * k + lane] = my_id;
-            warp_cnt[warp * E + my_id] = c + 1;
-        }
-        __syncwarp();
+        if (j == 0) top = bv;
+        ++nsel;
     }
-    __syncthreads();
-    // per expert: exclusive prefix over warps (warp order = token order)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int ww = 0; ww < kWarps; ++ww) {
-            const int c = warp_cnt[ww * E + e];
-            warp_cnt[ww * E + e] = run;
-            run += c;
-        }
-        block_hist[static_cast<int64_t>(blockIdx.x) * E + e] = run;
-    }
-    __syncthreads();
-    for (int q = threadIdx.x; q < kRouteTokensPerBlock * k; q += blockDim.x) {
-        const int id = s_id[q];
-        if (id < 0) continue;
-        const int tl = q / k;
-        local_rank[blk_tok0 * k + q] = warp_cnt[(tl / kTokPerWarp) * E + id] + s_rank[q];
+    const float ex = (lane < nsel) ? expf(my_val - top) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+    if (lane < k) {
+        ids[lane] = (lane < nsel) ? my_id : -1;
+        w[lane] = (lane < nsel) ? __fdiv_rn(ex, sum) : 0.0f;
     }
 }
 
-__global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ block_hist, int nblocks, int E,
-                                                          int32_t* __restrict__ offsets)
+// Blocks [0, n_topk): one token per warp.  Blocks [n_topk, gridDim.x): the
+// activation quantiser (optional).  Block 0 also resets the rank kernel's
+// arrival counter (this launch precedes it in stream order).
+template <int VPL>
+__global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float* __restrict__ logits, int64_t T,
+                                                                     int E, int k, int32_t* __restrict__ ids,
+                                                                     float* __restrict__ w, int* __restrict__ arrivals,
+                                                                     int64_t n_topk, const uint4* __restrict__ qx,
+                                                                     int64_t q_groups, uint8_t* __restrict__ q_codes,
+                                                                     float* __restrict__ q_scales)
 {
+    if (blockIdx.x >= n_topk) {
+        quant::groups(qx, q_groups, q_codes, q_scales, blockIdx.x - n_topk, gridDim.x - n_topk);
+        return;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *arrivals = 0;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5);
+    if (t >= T) return;
+    topk_token<VPL>(logits + t * E, E, k, ids + t * k, w + t * k, lane);
+}
+
+// One block per kRouteTokensPerBlock tokens; pairs of the block are taken
+// in rounds of kRankThreads (one per thread, in pair order).
+__global__ void __launch_bounds__(kRankThreads) route_rank_kernel(const int32_t* __restrict__ ids, int64_t T, int E,
+                                                                  int k, int32_t* __restrict__ block_hist,
+                                                                  int32_t* __restrict__ local_rank,
+                                                                  int* __restrict__ arrivals,
+                                                                  int32_t* __restrict__ offsets)
+{
+    extern __shared__ int32_t sm[];
+    int32_t* cnt = sm;                         // [32 warps][E]
+    int32_t* base = sm + 32 * E;               // [E] pairs of each expert in earlier rounds
+    __shared__ int s_last;
     __shared__ int32_t wsum[32];
-    const int e = threadIdx.x;
-    const int lane = e & 31, warp = e >> 5;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock;
+    const int64_t ntok = (T - t0) < kRouteTokensPerBlock ? (T - t0) : kRouteTokensPerBlock;
+    const int npairs = static_cast<int>(ntok) * k;
+    const int64_t p0 = t0 * k;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) base[i] = 0;
+
+    for (int r0 = 0; r0 < npairs; r0 += kRankThreads) {
+        for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
+        __syncthreads();
+        const int q = r0 + threadIdx.x;
+        int id = (q < npairs) ? __ldg(ids + p0 + q) : -1;
+        if (id >= E) id = -1;  // cannot come from route_topk; never ranked
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, id);
+        const int rank_w = __popc(peers & lt_mask);
+        if (id >= 0 && rank_w == 0) cnt[warp * E + id] = __popc(peers);
+        __syncthreads();
+        // per expert: exclusive prefix over warps (warp order = pair order)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int run = base[e];
+            for (int ww = 0; ww < 32; ++ww) {
+                const int c = cnt[ww * E + e];
+                cnt[ww * E + e] = run;
+                run += c;
+            }
+            base[e] = run;
+        }
+        __syncthreads();
+        if (id >= 0) local_rank[p0 + q] = cnt[warp * E + id] + rank_w;
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[static_cast<int64_t>(blockIdx.x) * E + e] = base[e];
+
+    // Arrival: the last block scans every block's counts.
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(arrivals, 1) == static_cast<int>(gridDim.x) - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int nblocks = gridDim.x;
+    const int e = threadIdx.x;  // one thread per expert (E <= 1024)
     int run = 0;
     if (e < E) {
-        // batches of independent loads, then their running prefix
+        // batches of independent loads, then their running prefix; counts of
+        // the other blocks are read from L2 (written before their arrival)
         for (int b0 = 0; b0 < nblocks; b0 += 16) {
             int c[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                c[j] = (b0 + j < nblocks) ? block_hist[static_cast<int64_t>(b0 + j) * E + e] : 0;
+                c[j] = (b0 + j < nblocks) ? __ldcg(block_hist + static_cast<int64_t>(b0 + j) * E + e) : 0;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 if (b0 + j < nblocks) block_hist[static_cast<int64_t>(b0 + j) * E + e] = run;
@@ -190,7 +223,7 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ ids, int64_t P,
     if (p >= P) return;
     const int total = offsets[E];
     const int e = ids[p];
-    if (e >= 0) {
+    if (e >= 0 && e < E) {
         const int64_t b = (p / k) / kRouteTokensPerBlock;
         const int64_t pos = static_cast<int64_t>(offsets[e]) + block_hist[b * E + e] + local_rank[p];
         sorted_pairs[pos] = static_cast<int32_t>(p);
@@ -203,45 +236,55 @@ __global__ void zero_offsets_kernel(int32_t* offsets, int n)
     for (int i = threadIdx.x; i < n; i += blockDim.x) offsets[i] = 0;
 }
 
-template <int VPL>
-size_t topk_smem(int E, int k)
-{
-    return (static_cast<size_t>(kWarps) * E + 2ull * kRouteTokensPerBlock * k) * sizeof(int32_t);
-}
-
-template <int VPL>
-cudaError_t run_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* hist,
-                     int32_t* lrank, int nblocks, cudaStream_t s)
-{
-    const size_t smem = topk_smem<VPL>(E, k);
-    if (smem > 48 * 1024) {
-        cudaError_t err =
-            cudaFuncSetAttribute(route_topk_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-    }
-    route_topk_kernel<VPL><<<nblocks, kWarps * 32, smem, s>>>(logits, T, E, k, ids, w, hist, lrank);
-    return cudaGetLastError();
-}
+size_t rank_smem(int E) { return (33ull * E) * sizeof(int32_t); }
 
 }  // namespace
 
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* offsets,
-                         int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank, cudaStream_t s)
+                         int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank, int* arrivals,
+                         const QuantArgs* quant, cudaStream_t s)
 {
+    int64_t q_groups = 0, q_blocks = 0;
+    DeviceInfo di;
+    if (!device_info(&di)) return cudaErrorUnknown;
+    if (quant && quant->T > 0) {
+        q_groups = quant->T * (quant->H / 128);
+        q_blocks = quant::blocks_for(q_groups, di.sm_count);
+    }
     if (T == 0 || k == 0) {
         zero_offsets_kernel<<<1, 256, 0, s>>>(offsets, E + 1);
         cudaError_t err = cudaGetLastError();
-        if (err != cudaSuccess || T == 0) return err;
-        // top_k == 0: nothing is routed; ids/w/sorted_pairs are empty
-        return cudaSuccess;
+        if (err != cudaSuccess || q_blocks == 0) return err;
+        // top_k == 0 or T == 0: nothing is routed; ids/w/sorted_pairs are empty
+        route_topk_kernel<2><<<static_cast<int>(q_blocks), kTopkWarps * 32, 0, s>>>(
+            logits, 0, E, k, ids, w, arrivals, 0, reinterpret_cast<const uint4*>(quant->x), q_groups, quant->codes,
+            quant->scales);
+        return cudaGetLastError();
     }
-    const int nblocks = static_cast<int>(ceil_div64(T, kRouteTokensPerBlock));
-    cudaError_t err;
-    if (E <= 64) err = run_topk<2>(logits, T, E, k, ids, w, block_hist, local_rank, nblocks, s);
-    else if (E <= 256) err = run_topk<8>(logits, T, E, k, ids, w, block_hist, local_rank, nblocks, s);
-    else err = run_topk<32>(logits, T, E, k, ids, w, block_hist, local_rank, nblocks, s);
+    const int64_t n_topk = ceil_div64(T, kTopkWarps);
+    const int grid = static_cast<int>(n_topk + q_blocks);
+    const uint4* qx = quant ? reinterpret_cast<const uint4*>(quant->x) : nullptr;
+    uint8_t* qc = quant ? quant->codes : nullptr;
+    float* qs = quant ? quant->scales : nullptr;
+    if (E <= 64)
+        route_topk_kernel<2><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+                                                               q_groups, qc, qs);
+    else if (E <= 256)
+        route_topk_kernel<8><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+                                                               q_groups, qc, qs);
+    else
+        route_topk_kernel<32><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+                                                                q_groups, qc, qs);
+    cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    route_scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblocks, E, offsets);
+    const int nblocks = static_cast<int>(ceil_div64(T, kRouteTokensPerBlock));
+    const size_t smem = rank_smem(E);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(route_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+    }
+    route_rank_kernel<<<nblocks, kRankThreads, smem, s>>>(ids, T, E, k, block_hist, local_rank, arrivals, offsets);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const int64_t P = T * k;
     route_scatter_kernel<<<static_cast<int>(ceil_div64(P, 256)), 256, 0, s>>>(ids, P, k, E, block_hist, local_rank,
@@ -309,7 +352,8 @@ extern "C" int moe_route_noalloc(const float* logits, int64_t T, int E, int top_
     auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
     if (!al(logits) || !al(topk_ids) || !al(topk_w) || !al(expert_offsets) || !al(sorted_pairs))
         return MOE_ERR_ALIGNMENT;
-    // the same scratch layout moe_route uses inside its workspace
+    // the layout moe_route uses inside its workspace: the arrival counter in
+    // the first 256 bytes, then the block histograms and the pair ranks
     const int64_t nblocks = ceil_div64(T > 0 ? T : 1, kRouteTokensPerBlock);
     const size_t off_hist = 256;
     const size_t off_rank = align_up(off_hist + static_cast<size_t>(nblocks) * E * 4, 256);
@@ -332,10 +376,10 @@ extern "C" int moe_route_noalloc(const float* logits, int64_t T, int E, int top_
         return MOE_ERR_CUDA;
     }
     // Nothing in the array has to start at zero: every call writes the
-    // histograms and ranks it later reads.
+    // counter, histograms and ranks it later reads.
     err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
                        reinterpret_cast<int32_t*>(base + off_hist), reinterpret_cast<int32_t*>(base + off_rank),
-                       static_cast<cudaStream_t>(stream));
+                       reinterpret_cast<int*>(base), nullptr, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) {
         std::snprintf(g_noalloc_error, sizeof(g_noalloc_error), "launch: %s", cudaGetErrorString(err));
         return MOE_ERR_CUDA;

@@ -7,6 +7,7 @@
  *                    permutation of (token, slot) pairs by expert;
  *   moe_quant_act    BF16 rows -> E4M3 codes with one FP32 scale per
  *                    1x128 group;
+ *   moe_route_quant  the two above in one call (fused first launch);
  *   moe_grouped_ffn  grouped gate/up GEMM, unclamped SiLU(gate)*up,
  *                    requantisation of the intermediate, grouped down GEMM
  *                    whose epilogue writes routing-weighted FP32 slot rows;
@@ -136,16 +137,39 @@ MOE_API int moe_route(const float* logits, int64_t T, int E, int top_k,
               void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_quant -- moe_route and moe_quant_act in one call, the activation
+ * quantiser riding in the router's first launch (both read only their own
+ * inputs, so neither waits for the other).  This is the fused router chain
+ * of "Integration for GLM-4.6-FP8 and performance tune on H20" (gap table
+ * row 7: the chain of small router kernels launched as one).
+ *
+ *   logits, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, ws_bytes:
+ *       as for moe_route (the workspace is moe_route_workspace_bytes(T, E,
+ *       top_k)); E, top_k: as for moe_route;
+ *   x, H, codes, scales: as for moe_quant_act (x [T, H] BF16 bits read;
+ *       codes [T, H] uint8 and scales [T, H/128] FP32 written).
+ *
+ * Results are bit-identical to the two separate calls.  Errors: the union of
+ * both calls' argument checks, before anything is enqueued; then as
+ * moe_route.  Three kernel launches in total (moe_route alone takes three,
+ * moe_quant_act one).
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route_quant(const float* logits, const uint16_t* x, int64_t T, int H, int E, int top_k,
+                            int32_t* topk_ids, float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs,
+                            uint8_t* codes, float* scales, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_route_noalloc -- moe_route without a workspace argument.  The pages
  * have no counterpart: this entry point exists for callers that cannot
  * allocate device memory at all (for example code running inside another
  * runtime's execution hook, which owns and pre-plans every device byte, or
  * a latency-critical path that cannot afford the implicit synchronisation of
- * cudaMalloc).  It allocates nothing; the router's scratch (block histograms
- * and per-pair ranks) lives in one static device array of 1 MiB + 4 KiB that
- * every GPU loading the library holds until the process exits.
+ * cudaMalloc).  It allocates nothing; the router's scratch (an arrival
+ * counter, block histograms and per-pair ranks) lives in one static device
+ * array of 1 MiB + 4 KiB that every GPU loading the library holds until the
+ * process exits.
  *   - Same arguments, results and limits as moe_route, and additionally the
- *     scratch of (T, E, top_k) must fit the array: ceil(T/128)*E*4 +
+ *     scratch of (T, E, top_k) must fit the array: 256 + ceil(T/128)*E*4 +
  *     T*top_k*4 bytes plus alignment (T = 16384, E = 1024, top_k = 8 fits).
  *     Larger requests return MOE_ERR_WORKSPACE before anything is enqueued;
  *     moe_route_noalloc_error() then names the sizes.

@@ -81,3 +81,66 @@ def test_route_rejects_bad_args():
     with pytest.raises(fm.MoeError) as e:
         fm.moe_route(lg, 2, z, z, z, z, ws[:8])  # workspace too small
     assert e.value.code == 4
+
+
+def _route_quant(logits, x, k):
+    T, E = logits.shape
+    H = x.shape[1]
+    ids = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), -7.0, dtype=torch.float32, device="cuda")
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    sp = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
+    codes = torch.full((T, H), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((T, H // 128), -7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty((fm.moe_route_workspace_bytes(T, E, k),), dtype=torch.uint8, device="cuda")
+    fm.moe_route_quant(logits, x, k, ids, w, off, sp, codes, scales, ws)
+    torch.cuda.synchronize()
+    assert fm.moe_get_device_status(ws) == 0
+    return ids, w, off, sp[: T * k], codes, scales
+
+
+def _separate(logits, x, k):
+    T, E = logits.shape
+    H = x.shape[1]
+    ids = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), -7.0, dtype=torch.float32, device="cuda")
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    sp = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
+    codes = torch.full((T, H), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((T, H // 128), -7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty((fm.moe_route_workspace_bytes(T, E, k),), dtype=torch.uint8, device="cuda")
+    fm.moe_route(logits, k, ids, w, off, sp, ws)
+    fm.moe_quant_act(x, codes, scales)
+    torch.cuda.synchronize()
+    return ids, w, off, sp[: T * k], codes, scales
+
+
+@pytest.mark.parametrize("T,H,E,k", [(0, 256, 8, 2), (37, 256, 8, 0), (1, 128, 1, 1), (333, 640, 64, 8),
+                                     (1000, 256, 1024, 32), (4096, 5120, 256, 8)])
+def test_route_quant_equals_separate_calls(T, H, E, k):
+    """The fused call (quantiser in the router's first launch) gives the
+    separate calls' results bit for bit, including the degenerate T = 0 and
+    top_k = 0 cases (top_k = 0 still quantises)."""
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + H + E + k)
+    lg = torch.randn((T, E), generator=g, device="cuda")
+    x = (torch.randn((T, H), generator=g, device="cuda") * 3).to(torch.bfloat16)
+    if T > 10:
+        x[3, 5] = float("nan")
+        x[4] = 0
+    a = _route_quant(lg, x, k)
+    b = _separate(lg, x, k)
+    for u, v, name in zip(a, b, ("ids", "w", "offsets", "sorted_pairs", "codes", "scales")):
+        assert torch.equal(u.view(torch.int32) if u.dtype == torch.float32 else u,
+                           v.view(torch.int32) if v.dtype == torch.float32 else v), name
+
+
+def test_route_quant_codes_match_oracle():
+    wl = mi.WORKLOADS["small"]
+    lg = mi.make_logits(wl, 0, "cuda")
+    x = mi.make_x(wl, 0, "cuda")
+    ids, w, off, sp, codes, scales = _route_quant(lg, x, wl.k)
+    rc, rs = oracle.quant_act(x.cpu())
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    rid, rw = oracle.route(lg.cpu(), wl.k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
