@@ -4,8 +4,9 @@
 // EXL3 on CUDA ...", commit text: routed FP32 rows).
 //
 // HBM-bound: each thread owns 4 consecutive columns of one token, reads the
-// token's slot ids (L1-resident), streams the valid slots' float4s and writes
-// one float4 (plus 8 bytes of BF16 when asked).  No atomics: the sum order is
+// token's slot ids (L1-resident), streams the valid slots' float4s (up to 8
+// loads in flight per thread) and writes one float4 (plus 8 bytes of BF16
+// when asked).  No atomics: the sum order is
 // the slot order, so a row's bits do not depend on other rows.
 // Algorithmic bytes per token: (#valid slots * H + H) * 4 (+ 2H for BF16).
 #include <cuda_bf16.h>
@@ -30,6 +31,8 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+constexpr int kSlotBatch = 8;  // slot rows loaded together per thread
+
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ ids,
                                                       int64_t T, int H4, int k, int E, float rs,
                                                       float4* __restrict__ out, uint2* __restrict__ out_bf16,
@@ -41,18 +44,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
         const int64_t t = i / H4;
         const int64_t c = i - t * H4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const int e = __ldg(ids + t * k + j);
-            if (e == -1) continue;
-            if (e < -1 || e >= E) {
-                if (c == 0) atomicOr(status, kDevBadExpertId);
-                continue;
+        // slots in batches: the batch's loads are all issued before the sums,
+        // which then run in slot order over the valid slots only
+        for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
+            float4 v[kSlotBatch];
+            bool ok[kSlotBatch];
+#pragma unroll
+            for (int u = 0; u < kSlotBatch; ++u) {
+                const int j = j0 + u;
+                const int e = (j < k) ? __ldg(ids + t * k + j) : -1;
+                if ((e < -1 || e >= E) && c == 0) atomicOr(status, kDevBadExpertId);
+                ok[u] = e >= 0 && e < E;
+                v[u] = ok[u] ? ld_stream_f4(y + (t * k + j) * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            const float4 v = ld_stream_f4(y + (t * k + j) * H4 + c);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+#pragma unroll
+            for (int u = 0; u < kSlotBatch; ++u) {
+                if (!ok[u]) continue;
+                acc.x += v[u].x;
+                acc.y += v[u].y;
+                acc.z += v[u].z;
+                acc.w += v[u].w;
+            }
         }
         const float4 o = make_float4(rs * acc.x, rs * acc.y, rs * acc.z, rs * acc.w);
         out[i] = o;

@@ -584,7 +584,17 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
         const int64_t t = pair / k;
         const uint4* src = reinterpret_cast<const uint4*>(codes + t * H);
         uint4* dst = reinterpret_cast<uint4*>(a_sorted + r * H);
-        for (int c = lane; c < H / 16; c += 32) dst[c] = __ldg(src + c);
+        // four 16-byte loads in flight per lane, then their stores
+        const int n16 = H / 16;
+        for (int c0 = lane; c0 < n16; c0 += 4 * 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c0 + 32 * u < n16) v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c0 + 32 * u < n16) dst[c0 + 32 * u] = v[u];
+        }
         for (int c = lane; c < GH; c += 32) sa_sorted[r * GH + c] = __ldg(act_scales + t * GH + c);
     }
 }

@@ -8,7 +8,7 @@
 // A half-warp owns one group: each lane loads one 16-byte vector (8 BF16),
 // the 16 lanes reduce amax with shuffles, each lane stores 8 code bytes, lane
 // 0 of the half stores the scale.  Loads are fully coalesced (a warp reads
-// 512 contiguous bytes), stores 256 contiguous bytes.
+// 512 contiguous bytes per group pair), stores 256 contiguous bytes.
 #pragma once
 
 #include "sm100.cuh"
@@ -25,8 +25,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p)
     return v;
 }
 
+constexpr int kUnroll = 4;  // groups per half-warp per trip, loads issued together
+
 // Quantises groups [0, n_groups) with the warps of `nblocks` blocks of
-// blockDim.x threads, this thread belonging to block `block`.
+// blockDim.x threads, this thread belonging to block `block`.  Per trip a
+// warp covers 2*kUnroll consecutive groups; its loads are issued before any
+// of them is reduced, so each lane keeps kUnroll 16-byte loads in flight.
 __device__ __forceinline__ void groups(const uint4* __restrict__ x, int64_t n_groups, uint8_t* __restrict__ codes,
                                        float* __restrict__ scales, int64_t block, int64_t nblocks)
 {
@@ -36,55 +40,62 @@ __device__ __forceinline__ void groups(const uint4* __restrict__ x, int64_t n_gr
     const int64_t warp = (block * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (nblocks * blockDim.x) >> 5;
 
-    for (int64_t g0 = warp * 2; g0 < n_groups; g0 += nwarps * 2) {
-        const int64_t g = g0 + half;
-        const bool active = g < n_groups;
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        if (active) raw = ld_stream(x + g * 16 + sub);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        float v[8];
+    for (int64_t g0 = warp * 2 * kUnroll; g0 < n_groups; g0 += nwarps * 2 * kUnroll) {
+        uint4 raw[kUnroll];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float(w[i] << 16);
-            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-        float amax = 0.0f;
-        int bad = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (isfinite(v[i])) amax = fmaxf(amax, fabsf(v[i]));
-            else bad = 1;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + 2 * u + half;
+            raw[u] = (g < n_groups) ? ld_stream(x + g * 16 + sub) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-            bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
-        }
-        float s = __fdiv_rn(amax, 448.0f);
-        if (s == 0.0f) s = 1.0f;
-        uint2 out;
-        if (bad) {
-            s = __int_as_float(0x7FC00000);
-            out = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        } else {
-            uint32_t p[4];
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t g = g0 + 2 * u + half;
+            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            float v[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                p[i] = sm100::e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
-            out = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
-        }
-        if (active) {
-            *reinterpret_cast<uint2*>(codes + g * 128 + sub * 8) = out;
-            if (sub == 0) scales[g] = s;
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = __uint_as_float(w[i] << 16);
+                v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            }
+            float amax = 0.0f;
+            int bad = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (isfinite(v[i])) amax = fmaxf(amax, fabsf(v[i]));
+                else bad = 1;
+            }
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) {
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+                bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
+            }
+            float s = __fdiv_rn(amax, 448.0f);
+            if (s == 0.0f) s = 1.0f;
+            uint2 out;
+            if (bad) {
+                s = __int_as_float(0x7FC00000);
+                out = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
+            } else {
+                uint32_t p[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    p[i] = sm100::e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
+                out = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+            }
+            if (g < n_groups) {
+                *reinterpret_cast<uint2*>(codes + g * 128 + sub * 8) = out;
+                if (sub == 0) scales[g] = s;
+            }
         }
     }
 }
 
-// Blocks of 256 threads that quantise n_groups: two groups per warp per
-// iteration, a few waves of 8 resident blocks per SM, grid-stride beyond.
+// Blocks of 256 threads that quantise n_groups: one trip of every warp over
+// the groups when the grid allows it, at most a few waves of 8 resident
+// blocks per SM (grid-stride beyond that).
 inline int64_t blocks_for(int64_t n_groups, int sm_count)
 {
-    const int64_t want = (n_groups + 15) / 16;
+    const int64_t want = (n_groups + 8 * 2 * kUnroll - 1) / (8 * 2 * kUnroll);
     const int64_t cap = static_cast<int64_t>(sm_count) * 8 * 4;
     return want < cap ? want : cap;
 }
