@@ -286,17 +286,20 @@ def main():
                          wl.k, wl.routed_scaling, wl.T)
     s = torch.cuda.current_stream()
 
-    # events: 7 per step (quantise, route, gather, gate/up, down, combine, end)
-    def mk():
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(s)
-        return e
-
-    evs = [[mk() for _ in range(7)] for _ in range(args.steps)]
+    # The product path: the layer captured once into a CUDA graph (the C
+    # ABI's moe_layer_plan) over resident input buffers, replayed per step.
+    x_in = torch.empty_like(d["x"])
+    lg_in = torch.empty_like(d["logits"])
+    x_in.copy_(d["x"])
+    lg_in.copy_(d["logits"])
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    plan = fm.LayerPlan(x_in, lg_in, wl.k, d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"],
+                        d["s_down"], wl.routed_scaling, stage_events=stage_ev)
     for _ in range(args.warmup):
         layer.forward(d["x"], d["logits"])
+        plan.launch()
     torch.cuda.synchronize()
-    if layer.device_status() != 0:
+    if layer.device_status() != 0 or plan.device_status() != 0:
         raise RuntimeError("device status reported a fault during warm-up")
     uuid = None
     try:
@@ -313,20 +316,41 @@ def main():
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(s)
     for i in range(args.steps):
-        layer.forward(d["x"], d["logits"], stage_events=evs[i])
+        plan.launch()
     t1.record(s)
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop() if sampler else None
     ms_total = max_over_ranks(world, t0.elapsed_time(t1))
     ms_step = ms_total / args.steps
-    status = layer.device_status()
-    # forward's events: 0 start, (1 = 0 when fused), 2 gather, 3 gate/up,
-    # 4 down, 5 combine, 6 end
-    spans = {"route_quant": (0, 2), "gather": (2, 3), "gemm_gateup": (3, 4), "gemm_down": (4, 5),
-             "combine": (5, 6)}
-    stage_ms = {n: statistics.mean(evs[i][a].elapsed_time(evs[i][b]) for i in range(args.steps))
-                for n, (a, b) in spans.items()}
+    # the graph's event nodes hold the last timed replay's marks
+    spans = {"route_quant": (0, 1), "gather": (1, 2), "gemm_gateup": (2, 3), "gemm_down": (3, 4),
+             "combine": (4, 5)}
+    last_ms = {n: stage_ev[a].elapsed_time(stage_ev[b]) for n, (a, b) in spans.items()}
+    status = plan.device_status()
+
+    # Per-stage averages from the events inside the graph (one launch at a
+    # time, after the timed region), and the same layer through the three
+    # separate calls.
+    acc = {n: [] for n in spans}
+    for _ in range(args.steps):
+        plan.launch()
+        torch.cuda.synchronize()
+        for n, (a, b) in spans.items():
+            acc[n].append(stage_ev[a].elapsed_time(stage_ev[b]))
+    stage_ms = {n: statistics.mean(v) for n, v in acc.items()}
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    c0.record(s)
+    for _ in range(args.steps):
+        layer.forward(d["x"], d["logits"])
+    c1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_calls = max_over_ranks(world, c0.elapsed_time(c1)) / args.steps
+    status |= layer.device_status()
 
     # roofline of the dominant kernel
     pk = peaks()
@@ -334,7 +358,7 @@ def main():
     P = int(off[-1])
     active = int(((off[1:] - off[:-1]) > 0).sum())
     gu_bytes = gateup_alg_bytes(wl, active, P)
-    gu_s = stage_ms["gemm_gateup"] / 1e3
+    gu_s = last_ms["gemm_gateup"] / 1e3
     achieved = gu_bytes / gu_s / 1e9
     flops = mi.flops_per_layer(wl, P)
     gemm_s = (stage_ms["gemm_gateup"] + stage_ms["gemm_down"]) / 1e3
@@ -348,21 +372,19 @@ def main():
     x_h = d["x"].cpu().pin_memory()
     lg_h = d["logits"].cpu().pin_memory()
     out_h = torch.empty((wl.T, wl.H), dtype=torch.float32).pin_memory()
-    x_d = torch.empty_like(d["x"])
-    lg_d = torch.empty_like(d["logits"])
     for _ in range(2):
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        out_h.copy_(layer.forward(x_d, lg_d), non_blocking=True)
+        x_in.copy_(x_h, non_blocking=True)
+        lg_in.copy_(lg_h, non_blocking=True)
+        out_h.copy_(plan.launch(), non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s)
     for _ in range(args.steps):
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        out_h.copy_(layer.forward(x_d, lg_d), non_blocking=True)
+        x_in.copy_(x_h, non_blocking=True)
+        lg_in.copy_(lg_h, non_blocking=True)
+        out_h.copy_(plan.launch(), non_blocking=True)
     e1.record(s)
     torch.cuda.synchronize()
     barrier(world)
@@ -396,6 +418,8 @@ def main():
                              "fp8_peak_tflops": fp8_peak, "roofline_ms": roof_s * 1e3,
                              "frac_roofline": roof_s / gemm_s},
             "stages_ms": stage_ms,
+            "stages_ms_last_timed_step": last_ms,
+            "ms_per_step_three_calls": ms_calls,
             "e2e": {"value": whole_job_tokens_per_s(world, wl.T, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                     "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms},
@@ -409,6 +433,7 @@ def main():
         if clocks:
             line["clocks"] = clocks
         print(json.dumps(line), flush=True)
+    plan.close()
     if world > 1:
         torch.distributed.destroy_process_group()
 

@@ -61,6 +61,19 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc_error.argtypes = []
         L.moe_quant_act.restype = i32
         L.moe_quant_act.argtypes = [P, i64, i32, P, P, P]
+        L.moe_layer_workspace_bytes.restype = sz
+        L.moe_layer_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+        L.moe_layer.restype = i32
+        L.moe_layer.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, P, ctypes.c_float, P, P, P, sz, P]
+        L.moe_layer_plan_create.restype = i32
+        L.moe_layer_plan_create.argtypes = [ctypes.POINTER(ctypes.c_void_p), P, P, i64, i32, i32, i32, i32,
+                                            P, P, P, P, P, P, ctypes.c_float, P, P, P, sz, P]
+        L.moe_layer_plan_launch.restype = i32
+        L.moe_layer_plan_launch.argtypes = [P, P]
+        L.moe_layer_plan_destroy.restype = None
+        L.moe_layer_plan_destroy.argtypes = [P]
+        L.moe_layer_get_device_status.restype = i32
+        L.moe_layer_get_device_status.argtypes = [P, i64, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int)]
         L.moe_route_quant.restype = i32
         L.moe_route_quant.argtypes = [P, P, i64, i32, i32, i32, P, P, P, P, P, P, P, sz, P]
         L.moe_ffn_workspace_bytes.restype = sz
@@ -201,6 +214,79 @@ def moe_ffn_intermediate(ws, T: int, H: int, I: int, top_k: int):
     codes = ws[oc: oc + P * GI * 128].view(P, GI * 128)
     scales = ws[osc: osc + P * GI * 4].view(torch.float32).view(P, GI)
     return codes, scales
+
+
+def moe_layer_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> int:
+    return int(lib().moe_layer_workspace_bytes(T, H, I, E, top_k))
+
+
+def moe_layer(logits, x, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling, out_f32, out_bf16, ws,
+              stream=None):
+    """The whole layer (moe_route_quant, moe_grouped_ffn, moe_combine) over
+    one workspace of moe_layer_workspace_bytes."""
+    T, E = logits.shape
+    H = x.shape[1]
+    I = w_gate.shape[1]
+    _check(lib().moe_layer(_p(logits), _p(x), T, H, E, top_k, I, _p(w_gate), _p(s_gate), _p(w_up), _p(s_up),
+                           _p(w_down), _p(s_down), routed_scaling, _p(out_f32), _p(out_bf16), _p(ws),
+                           ws.numel() * ws.element_size(), _s(stream)), "moe_layer")
+
+
+def moe_layer_get_device_status(ws, T: int, H: int, I: int, E: int, top_k: int) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().moe_layer_get_device_status(_p(ws), T, H, I, E, top_k, ctypes.byref(v)),
+           "moe_layer_get_device_status")
+    return v.value
+
+
+class LayerPlan:
+    """The layer captured into a CUDA graph for fixed buffers (the C ABI's
+    moe_layer_plan).  ``x`` and ``logits`` are the input buffers the graph
+    reads and ``out`` the FP32 rows it writes; copy each batch into ``x`` and
+    ``logits`` before ``launch``.  The plan owns its workspace."""
+
+    def __init__(self, x, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling,
+                 out_bf16=None, stage_events=None):
+        T, E = logits.shape
+        H = x.shape[1]
+        I = w_gate.shape[1]
+        self.shape = (T, H, I, E, int(top_k))
+        self.x, self.logits = x, logits
+        self.w = (w_gate, s_gate, w_up, s_up, w_down, s_down)
+        self.out = torch.empty((T, H), dtype=torch.float32, device=x.device)
+        self.out_bf16 = out_bf16
+        self.ws = torch.empty((moe_layer_workspace_bytes(T, H, I, E, top_k),), dtype=torch.uint8, device=x.device)
+        self.events = stage_events
+        evs = None
+        if stage_events is not None:
+            assert len(stage_events) == 6
+            for e in stage_events:
+                if not e.cuda_event:  # torch creates the CUDA event at its first record
+                    e.record()
+            evs = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
+        h = ctypes.c_void_p(0)
+        _check(lib().moe_layer_plan_create(ctypes.byref(h), _p(logits), _p(x), T, H, E, int(top_k), I,
+                                           *[_p(t) for t in self.w], float(routed_scaling), _p(self.out),
+                                           _p(out_bf16), _p(self.ws), self.ws.numel(), evs), "moe_layer_plan_create")
+        self._h = h
+
+    def launch(self, stream=None) -> torch.Tensor:
+        _check(lib().moe_layer_plan_launch(self._h, _s(stream)), "moe_layer_plan_launch")
+        return self.out
+
+    def device_status(self) -> int:
+        return moe_layer_get_device_status(self.ws, *self.shape)
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            lib().moe_layer_plan_destroy(self._h)
+            self._h = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ------------------------------------------------------------------ layer

@@ -681,7 +681,7 @@ namespace {
 cudaError_t stage_mark(const FfnArgs& a, int i, cudaStream_t s)
 {
     if (!a.stage_events || !a.stage_events[i]) return cudaSuccess;
-    return cudaEventRecord(static_cast<cudaEvent_t>(a.stage_events[i]), s);
+    return record_event(a.stage_events[i], s);
 }
 }  // namespace
 

@@ -19,6 +19,19 @@ constexpr int kDevWaitTimeout = 0x8;
 constexpr int kRouteTokensPerBlock = 128;
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Records a caller's timing event on s.  Inside a stream capture a plain
+// record only orders the capture; the external flag makes it an event node
+// that records on every replay of the graph.
+inline cudaError_t record_event(void* ev, cudaStream_t s)
+{
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t err = cudaStreamIsCapturing(s, &cap);
+    if (err != cudaSuccess) return err;
+    return cap == cudaStreamCaptureStatusActive
+               ? cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), s, cudaEventRecordExternal)
+               : cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
+}
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct DeviceInfo {

@@ -281,6 +281,55 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_layer -- the whole routed-expert layer in one call: moe_route_quant,
+ * moe_grouped_ffn and moe_combine, stream-ordered, over one caller
+ * workspace that also holds the intermediates (codes, scales, routing,
+ * permutation, slot rows y).  Results are those of the three calls.
+ *
+ *   logits [T, E] FP32, x [T, H] BF16 bits: read;
+ *   w_* / s_*: as for moe_grouped_ffn; routed_scaling, out_f32 [T, H],
+ *   out_bf16 (nullable): as for moe_combine;
+ *   ws, ws_bytes: at least moe_layer_workspace_bytes(T, H, I, E, top_k).
+ *
+ * Errors: as the three calls (the first failing one's status is returned;
+ * the calls before it stay enqueued).  Limits: the three calls' limits, and
+ * top_k >= 1.
+ *
+ * moe_layer_plan_create captures the same sequence for fixed pointers and
+ * sizes into a CUDA graph (thread-local stream capture on a private stream;
+ * nothing runs at creation) and instantiates it.  moe_layer_plan_launch
+ * enqueues the graph on `stream`: one launch per layer instead of seven
+ * kernel launches, three status memsets and the host-side checks.  The
+ * plan reads its inputs from, and writes its outputs to, the addresses given
+ * at creation, so a caller copies each batch into them.  stage_events
+ * (nullable) are 6 cudaEvent_t recorded inside the graph at the start,
+ * before the gather, gate/up and down launches, after the down launch, and
+ * at the end.  A plan belongs to the device current at creation; destroy it
+ * before its buffers.  One plan's launches must not overlap each other.
+ * The pages' counterpart: the router chain and the layer captured in-graph
+ * ("Integration for GLM-4.6-FP8 and performance tune on H20", gap table
+ * row 7).
+ *
+ * moe_layer_get_device_status: synchronous; ORs the status words of the
+ * three calls held in a layer workspace (moe_get_device_status semantics).
+ * ------------------------------------------------------------------------- */
+typedef struct moe_layer_plan moe_layer_plan;
+MOE_API size_t moe_layer_workspace_bytes(int64_t T, int H, int I, int E, int top_k);
+MOE_API int moe_layer(const float* logits, const uint16_t* x, int64_t T, int H, int E, int top_k, int I,
+                      const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up, const float* s_up,
+                      const uint8_t* w_down, const float* s_down, float routed_scaling,
+                      float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes, void* stream);
+MOE_API int moe_layer_plan_create(moe_layer_plan** plan, const float* logits, const uint16_t* x, int64_t T,
+                                  int H, int E, int top_k, int I, const uint8_t* w_gate, const float* s_gate,
+                                  const uint8_t* w_up, const float* s_up, const uint8_t* w_down,
+                                  const float* s_down, float routed_scaling, float* out_f32, uint16_t* out_bf16,
+                                  void* ws, size_t ws_bytes, void* const* stage_events);
+MOE_API int moe_layer_plan_launch(moe_layer_plan* plan, void* stream);
+MOE_API void moe_layer_plan_destroy(moe_layer_plan* plan);
+MOE_API int moe_layer_get_device_status(const void* ws, int64_t T, int H, int I, int E, int top_k,
+                                        int* status_out);
+
+/* ---------------------------------------------------------------------------
  * moe_get_device_status -- synchronously read the
  * status word at the start of a workspace used by moe_route,
  * moe_grouped_ffn or moe_combine.  Waits for all work on the device.
