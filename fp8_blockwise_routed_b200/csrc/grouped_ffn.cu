@@ -16,7 +16,9 @@
 //              128 up) columns, one MMA of N=256 per 32-wide K step; epilogue
 //              h = SiLU(g)*u, requantised per 128-group -> h codes/scales
 //   down     : same kernel, tile = 128 rows x 256 output columns over the
-//              intermediate; epilogue y[pair] = w_pair * o
+//              intermediate; epilogue y[pair] = w_pair * o, each 256-byte row
+//              segment staged in shared memory and written by a bulk copy
+//              (3 weight stages; the rest of the ring holds the staging)
 //
 // Block scales (FP32, not powers of two) have no tensor-core path, so every
 // 128-deep K block is its own MMA chain into a fresh TMEM accumulator
@@ -61,7 +63,8 @@ using namespace sm100;
 constexpr int BM = 128;
 constexpr int BK = 128;
 constexpr int A_STAGES = 3;               // activation tiles: L2 hits, short latency
-constexpr int B_STAGES = 5;               // weight tiles: streamed from HBM, long latency
+constexpr int B_STAGES = 5;               // weight tiles (gate/up): streamed from HBM, long latency
+constexpr int B_STAGES_DOWN = 3;          // weight tiles (down): the rest of the ring stages y rows
 constexpr int A_TILE = BM * BK;           // 16 KiB
 constexpr int B_HALF = 128 * BK;          // 16 KiB
 constexpr int B_TILE = 2 * B_HALF;        // 32 KiB
@@ -83,7 +86,17 @@ constexpr int MAX_E = 1024;
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + A_STAGES * A_TILE;
-constexpr int OFF_BARS = OFF_B + B_STAGES * B_TILE;
+// down: each epilogue thread stages its 64-column y segment (256 B) here for
+// a bulk copy to global memory; slots 272 B apart so a warp's 16-byte shared
+// stores spread over all banks
+constexpr int STAGE_SLOT = 272;
+constexpr int OFF_STAGE = OFF_B + B_STAGES_DOWN * B_TILE;
+constexpr int STAGE_BYTES = EPI_WARPS * 32 * STAGE_SLOT;
+constexpr int RING_BYTES =
+    B_STAGES * B_TILE > B_STAGES_DOWN * B_TILE + STAGE_BYTES ? B_STAGES * B_TILE : B_STAGES_DOWN * B_TILE + STAGE_BYTES;
+constexpr int OFF_BARS = OFF_B + RING_BYTES;
+template <int MODE>
+constexpr int b_stages() { return MODE == 0 ? B_STAGES : B_STAGES_DOWN; }
 // barriers: fullA, emptyA, fullB, emptyB, tfull[2], tempty[2], xbar[4]
 constexpr int BAR_FULL_A = 0;
 constexpr int BAR_EMPTY_A = BAR_FULL_A + A_STAGES;
@@ -122,7 +135,6 @@ struct GemmParams {
     const int32_t* sorted_pairs;
     const float* topk_w;
     float* y;              // [P, H]
-    int y_v8;              // y is 32-byte aligned: 32-byte stores
     int H;
     int* status;
 };
@@ -166,6 +178,7 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
                                            const int* seg, const int* ipre, int total_items, uint32_t sbase,
                                            uint32_t bars, volatile int* abort)
 {
+    constexpr int BS = b_stages<MODE>();
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
@@ -173,8 +186,8 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
         const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
         const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-            const int s = it % B_STAGES;
-            if (!mbar_wait_bounded(bars + 8 * (BAR_EMPTY_B + s), ((it / B_STAGES) & 1) ^ 1, abort, WAIT_NS)) {
+            const int s = it % BS;
+            if (!mbar_wait_bounded(bars + 8 * (BAR_EMPTY_B + s), ((it / BS) & 1) ^ 1, abort, WAIT_NS)) {
                 ok = false;
                 break;
             }
@@ -186,9 +199,9 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
         }
     }
     if (!ok) {  // let the copies already issued land before the CTA can exit
-        for (int j = it - B_STAGES > 0 ? it - B_STAGES : 0; j < it; ++j) {
+        for (int j = it - BS > 0 ? it - BS : 0; j < it; ++j) {
             volatile int no_abort = 0;
-            mbar_wait_bounded(bars + 8 * (BAR_FULL_B + j % B_STAGES), (j / B_STAGES) & 1, &no_abort, WAIT_NS / 4);
+            mbar_wait_bounded(bars + 8 * (BAR_FULL_B + j % BS), (j / BS) & 1, &no_abort, WAIT_NS / 4);
         }
     }
 }
@@ -229,20 +242,22 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
 // block is promoted with its own scales), then commits that free the A and B
 // stages and hand the buffer to the epilogue.  A commit tracks the MMAs of
 // the issuing thread only, which are exactly the ones it hands over.
+template <int MODE>
 __device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars,
                                          uint32_t tmem, volatile int* abort, int parity)
 {
+    constexpr int BS = b_stages<MODE>();
     constexpr uint32_t idesc = idesc_e4m3_f32(128, 256);
     int it = 0;
     int last_commit = -1;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             if ((it & 1) != parity) continue;  // the other issuer's K block
-            const int sa = it % A_STAGES, sb = it % B_STAGES, b = it & 1;
+            const int sa = it % A_STAGES, sb = it % BS, b = it & 1;
             // no tcgen05 fence after the TMEM wait: the epilogue released the
             // buffer only after tcgen05.wait::ld, so its reads are complete
             if (!mbar_spin_bounded(bars + 8 * (BAR_TEMPTY + b), ((it >> 1) & 1) ^ 1, abort, WAIT_NS) ||
-                !mbar_spin_bounded(bars + 8 * (BAR_FULL_B + sb), (it / B_STAGES) & 1, abort, WAIT_NS) ||
+                !mbar_spin_bounded(bars + 8 * (BAR_FULL_B + sb), (it / BS) & 1, abort, WAIT_NS) ||
                 !mbar_spin_bounded(bars + 8 * (BAR_FULL_A + sa), (it / A_STAGES) & 1, abort, WAIT_NS))
                 goto drain;
             {
@@ -430,37 +445,26 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                     float* dst = p.y + static_cast<int64_t>(pair) * p.H;
                     const int c0 = w.nt * 256 + half * 64;
                     const int c1 = c0 + 128;
-                    // 32-byte stores (whole sectors) when y allows, else 16-byte
-                    if (p.y_v8) {
-                        if (c0 < p.H) {
+                    // Each 64-column segment (256 contiguous bytes of the
+                    // pair's y row) goes through this thread's shared slot
+                    // to a bulk copy, so the TMA engine does the global
+                    // writes while the warp returns to the next item.  The
+                    // slot is rewritten only after the copies that read it
+                    // have done so.
+                    const uint32_t slot = bars - OFF_BARS + OFF_STAGE + (threadIdx.x - 128) * STAGE_SLOT;
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                st_global_v8(dst + c0 + 8 * c, wt * acc0[8 * c], wt * acc0[8 * c + 1],
-                                             wt * acc0[8 * c + 2], wt * acc0[8 * c + 3], wt * acc0[8 * c + 4],
-                                             wt * acc0[8 * c + 5], wt * acc0[8 * c + 6], wt * acc0[8 * c + 7]);
-                        }
-                        if (c1 < p.H) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int c = hh ? c1 : c0;
+                        if (c >= p.H) continue;
+                        const float* a = hh ? acc1 : acc0;
+                        bulk_wait_read_all();
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                st_global_v8(dst + c1 + 8 * c, wt * acc1[8 * c], wt * acc1[8 * c + 1],
-                                             wt * acc1[8 * c + 2], wt * acc1[8 * c + 3], wt * acc1[8 * c + 4],
-                                             wt * acc1[8 * c + 5], wt * acc1[8 * c + 6], wt * acc1[8 * c + 7]);
-                        }
-                    } else {
-                        if (c0 < p.H) {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c)
-                                reinterpret_cast<float4*>(dst + c0)[c] =
-                                    make_float4(wt * acc0[4 * c], wt * acc0[4 * c + 1], wt * acc0[4 * c + 2],
-                                                wt * acc0[4 * c + 3]);
-                        }
-                        if (c1 < p.H) {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c)
-                                reinterpret_cast<float4*>(dst + c1)[c] =
-                                    make_float4(wt * acc1[4 * c], wt * acc1[4 * c + 1], wt * acc1[4 * c + 2],
-                                                wt * acc1[4 * c + 3]);
-                        }
+                        for (int q4 = 0; q4 < 16; ++q4)
+                            st_shared_v4(slot + 16 * q4, wt * a[4 * q4], wt * a[4 * q4 + 1], wt * a[4 * q4 + 2],
+                                         wt * a[4 * q4 + 3]);
+                        fence_proxy_async_smem();
+                        bulk_store(dst + c, slot, 256);
+                        bulk_commit();
                     }
                 }
             }
@@ -543,12 +547,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         setmaxnreg_dec<REGS_CTRL>();
         if ((threadIdx.x & 31) == 0) {
             if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
-            else if (warp == 1 || warp == 2) mma_role(p, total_items, sbase, bars, tmem, abort, warp - 1);
+            else if (warp == 1 || warp == 2) mma_role<MODE>(p, total_items, sbase, bars, tmem, abort, warp - 1);
             else if (warp == 3) producer_a(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {
         setmaxnreg_inc<REGS_EPI>();
         epilogue_role<MODE>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
+        // the y bulk copies must be done with shared memory (and complete)
+        // before the CTA exits
+        if (MODE == 1) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -760,7 +767,6 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     d.b_s1 = a.s_down;
     d.b_nblocks = GH;
     d.rev = 0;
-    d.y_v8 = (reinterpret_cast<uintptr_t>(a.y) & 31u) == 0;
     if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
     if ((err = run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;
     return stage_mark(a, 3, s);
