@@ -74,6 +74,17 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_plan_destroy.argtypes = [P]
         L.moe_layer_get_device_status.restype = i32
         L.moe_layer_get_device_status.argtypes = [P, i64, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int)]
+        L.moe_ep_plan_workspace_bytes.restype = sz
+        L.moe_ep_plan_workspace_bytes.argtypes = [i64, i32, i32]
+        L.moe_ep_plan.restype = i32
+        L.moe_ep_plan.argtypes = [P, i64, i32, i32, i32, i32, i64, P, P, P, P, P, P, sz, P]
+        L.moe_permute.restype = i32
+        L.moe_permute.argtypes = [P, i64, i32, i32, P, P, P, sz, P]
+        L.moe_grouped_ffn_rows.restype = i32
+        L.moe_grouped_ffn_rows.argtypes = [P, P, i64, i32, P, P, i32, P, P, i32, i32, P, P, P, P, P, P, P, P, i64,
+                                           P, sz, P, P]
+        L.moe_combine_rows.restype = i32
+        L.moe_combine_rows.argtypes = [P, i64, P, i64, i32, i32, ctypes.c_float, P, P, P, sz, P]
         L.moe_route_quant.restype = i32
         L.moe_route_quant.argtypes = [P, P, i64, i32, i32, i32, P, P, P, P, P, P, P, sz, P]
         L.moe_ffn_workspace_bytes.restype = sz
@@ -287,6 +298,45 @@ class LayerPlan:
             self.close()
         except Exception:
             pass
+
+
+def moe_ep_plan_workspace_bytes(T: int, top_k: int, world: int) -> int:
+    return int(lib().moe_ep_plan_workspace_bytes(T, top_k, world))
+
+
+def moe_ep_plan(topk_ids, num_experts, world, rank, T_home, local_ids, send_rows, recv_rows, offs_oh, offs_ho, ws,
+                stream=None):
+    T, k = topk_ids.shape
+    _check(lib().moe_ep_plan(_p(topk_ids), T, k, num_experts, world, rank, T_home, _p(local_ids), _p(send_rows),
+                             _p(recv_rows), _p(offs_oh), _p(offs_ho), _p(ws), ws.numel() * ws.element_size(),
+                             _s(stream)), "moe_ep_plan")
+
+
+def moe_permute(ids, num_experts, expert_offsets, sorted_pairs, ws, stream=None):
+    """The stable permutation of moe_route on caller-given ids [T, k]."""
+    T, k = ids.shape
+    _check(lib().moe_permute(_p(ids), T, num_experts, k, _p(expert_offsets), _p(sorted_pairs), _p(ws),
+                             ws.numel() * ws.element_size(), _s(stream)), "moe_permute")
+
+
+def moe_grouped_ffn_rows(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs, w_gate, s_gate, w_up,
+                         s_up, w_down, s_down, y, y_rows, ws, stream=None):
+    """moe_grouped_ffn writing pair p to row y_rows[p] of y (-1: not written)."""
+    T, H = codes.shape
+    k = topk_ids.shape[1]
+    E, I = w_gate.shape[0], w_gate.shape[1]
+    _check(lib().moe_grouped_ffn_rows(_p(codes), _p(act_scales), T, H, _p(topk_ids), _p(topk_w), k,
+                                      _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate), _p(w_up),
+                                      _p(s_up), _p(w_down), _p(s_down), _p(y), _p(y_rows), y.shape[0], _p(ws),
+                                      ws.numel() * ws.element_size(), _s(stream), None), "moe_grouped_ffn_rows")
+
+
+def moe_combine_rows(y, rows, routed_scaling, out_f32, out_bf16, ws, stream=None):
+    """out[t] = routed_scaling * sum_j y[rows[t, j]] over rows >= 0, slot order."""
+    T, k = rows.shape
+    H = out_f32.shape[1]
+    _check(lib().moe_combine_rows(_p(y), y.shape[0], _p(rows), T, H, k, routed_scaling, _p(out_f32), _p(out_bf16),
+                                  _p(ws), ws.numel() * ws.element_size(), _s(stream)), "moe_combine_rows")
 
 
 # ------------------------------------------------------------------ layer

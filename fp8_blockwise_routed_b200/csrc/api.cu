@@ -84,19 +84,9 @@ int clear_status(void* ws, cudaStream_t s)
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "status clear");
 }
 
-// Route workspace: status word, arrival counter (256 bytes), block histograms
-// [ceil(T/128), E] i32, pair ranks [T*k] i32.
 size_t route_layout(int64_t T, int E, int k, size_t* off_arr, size_t* off_hist, size_t* off_rank)
 {
-    const int64_t nblocks = ceil_div64(T > 0 ? T : 1, kRouteTokensPerBlock);
-    size_t o = kStatusBytes;
-    *off_arr = o;
-    o += 256;
-    *off_hist = o;
-    o = align_up(o + static_cast<size_t>(nblocks) * (E > 0 ? E : 1) * 4, 256);
-    *off_rank = o;
-    o = align_up(o + static_cast<size_t>(T > 0 ? T : 1) * (k > 0 ? k : 1) * 4, 256);
-    return o;
+    return route_ws_layout(T, E, k, off_arr, off_hist, off_rank);
 }
 
 }  // namespace
@@ -200,6 +190,20 @@ int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, in
                     const float* s_up, const uint8_t* w_down, const float* s_down, float* y, void* ws,
                     size_t ws_bytes, void* stream, void* const* stage_events)
 {
+    return moe_grouped_ffn_rows(codes, act_scales, T, H, topk_ids, topk_w, top_k, expert_offsets, sorted_pairs, E, I,
+                                w_gate, s_gate, w_up, s_up, w_down, s_down, y, nullptr, 0, ws, ws_bytes, stream,
+                                stage_events);
+}
+
+int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t T, int H, const int32_t* topk_ids,
+                         const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs,
+                         int E, int I, const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
+                         const float* s_up, const uint8_t* w_down, const float* s_down, float* y,
+                         const int32_t* y_rows, int64_t y_nrows, void* ws, size_t ws_bytes, void* stream,
+                         void* const* stage_events)
+{
+    if (y_rows && y_nrows < 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_rows)) return MOE_ERR_ALIGNMENT;
     if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOP_K) return MOE_ERR_INVALID_ARG;
     if (I < 1 || I > MOE_MAX_INTERMEDIATE) return MOE_ERR_INVALID_ARG;
@@ -239,6 +243,8 @@ int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, in
     a.w_down = w_down;
     a.s_down = s_down;
     a.y = y;
+    a.y_rows = y_rows;
+    a.y_nrows = y_nrows;
     a.status = reinterpret_cast<int*>(w8);
     a.a_sorted = w8 + off_a;
     a.sa_sorted = reinterpret_cast<float*>(w8 + off_sa);
@@ -266,6 +272,24 @@ int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int H, int t
     cudaError_t err = launch_combine(y, topk_ids, T, H, top_k, E, routed_scaling, out_f32, out_bf16,
                                      static_cast<int*>(ws), s);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
+}
+
+int moe_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int top_k,
+                     float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes, void* stream)
+{
+    if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (top_k < 0 || top_k > MOE_MAX_TOP_K || y_nrows < 0) return MOE_ERR_INVALID_ARG;
+    if (!ws || (T > 0 && !out_f32) || (T > 0 && top_k > 0 && (!rows || (y_nrows > 0 && !y))))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(rows) || !aligned16(out_f32) || !aligned16(out_bf16) || !aligned16(ws))
+        return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    if (int r = check_device()) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int r = clear_status(ws, s)) return r;
+    cudaError_t err = launch_combine_rows(y, y_nrows, rows, T, H, top_k, routed_scaling, out_f32, out_bf16,
+                                          static_cast<int*>(ws), s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine_rows");
 }
 
 int moe_get_device_status(const void* ws, int* status_out)

@@ -72,7 +72,62 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
     }
 }
 
+// The same sum with each slot's row taken from a row map (-1: empty slot).
+__global__ void __launch_bounds__(256) combine_rows_kernel(const float4* __restrict__ y, int64_t y_nrows,
+                                                           const int32_t* __restrict__ rows, int64_t T, int H4, int k,
+                                                           float rs, float4* __restrict__ out,
+                                                           uint2* __restrict__ out_bf16, int* __restrict__ status)
+{
+    const int64_t n = T * H4;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t t = i / H4;
+        const int64_t c = i - t * H4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
+            float4 v[kSlotBatch];
+            bool ok[kSlotBatch];
+#pragma unroll
+            for (int u = 0; u < kSlotBatch; ++u) {
+                const int j = j0 + u;
+                const int64_t row = (j < k) ? __ldg(rows + t * k + j) : -1;
+                if (row >= y_nrows && c == 0) atomicOr(status, kDevBadPair);
+                ok[u] = row >= 0 && row < y_nrows;
+                v[u] = ok[u] ? ld_stream_f4(y + row * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kSlotBatch; ++u) {
+                if (!ok[u]) continue;
+                acc.x += v[u].x;
+                acc.y += v[u].y;
+                acc.z += v[u].z;
+                acc.w += v[u].w;
+            }
+        }
+        const float4 o = make_float4(rs * acc.x, rs * acc.y, rs * acc.z, rs * acc.w);
+        out[i] = o;
+        if (out_bf16) out_bf16[i] = make_uint2(bf16x2_rn(o.x, o.y), bf16x2_rn(o.z, o.w));
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int k,
+                                float rs, float* out, uint16_t* out_bf16, int* status, cudaStream_t s)
+{
+    const int H4 = H / 4;
+    const int64_t n = T * H4;
+    if (n == 0) return cudaSuccess;
+    DeviceInfo di;
+    if (!device_info(&di)) return cudaErrorUnknown;
+    const int64_t want = ceil_div64(n, 256);
+    const int64_t cap = static_cast<int64_t>(di.sm_count) * 8 * 8;
+    const int grid = static_cast<int>(want < cap ? want : cap);
+    combine_rows_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), y_nrows, rows, T, H4, k, rs,
+                                             reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16),
+                                             status);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
                            float* out, uint16_t* out_bf16, int* status, cudaStream_t s)

@@ -134,7 +134,9 @@ struct GemmParams {
     // down epilogue
     const int32_t* sorted_pairs;
     const float* topk_w;
-    float* y;              // [P, H]
+    float* y;              // [P, H], or [y_nrows, H] rows through y_rows
+    const int32_t* y_rows; // nullable: y row of each pair (-1: not written)
+    int64_t y_nrows;
     int H;
     int* status;
 };
@@ -317,10 +319,14 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
         // down: the row's pair index and routing weight, fetched before the
         // K loop so that the tail does not wait on them
         int pair = -1;
+        int64_t yrow = -1;
         float wt = 0.f;
         if (MODE == 1 && valid) {
             pair = __ldg(p.sorted_pairs + r);
-            if (pair >= 0 && pair < p.P) wt = __ldg(p.topk_w + pair);
+            if (pair >= 0 && pair < p.P) {
+                wt = __ldg(p.topk_w + pair);
+                yrow = p.y_rows ? __ldg(p.y_rows + pair) : pair;
+            }
         }
 
         float acc0[64], acc1[64];
@@ -439,10 +445,10 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             }
         } else {
             if (valid) {
-                if (pair < 0 || pair >= p.P) {
+                if (pair < 0 || pair >= p.P || yrow >= p.y_nrows) {
                     atomicOr(p.status, kDevBadPair);
-                } else {
-                    float* dst = p.y + static_cast<int64_t>(pair) * p.H;
+                } else if (yrow >= 0) {
+                    float* dst = p.y + yrow * p.H;
                     const int c0 = w.nt * 256 + half * 64;
                     const int c1 = c0 + 128;
                     // Each 64-column segment (256 contiguous bytes of the
@@ -752,6 +758,8 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     g.sorted_pairs = a.sorted_pairs;
     g.topk_w = a.topk_w;
     g.y = a.y;
+    g.y_rows = a.y_rows;
+    g.y_nrows = a.y_rows ? a.y_nrows : P;
     g.H = H;
     g.status = a.status;
     if ((err = stage_mark(a, 1, s)) != cudaSuccess) return err;

@@ -19,6 +19,23 @@ constexpr int kDevWaitTimeout = 0x8;
 constexpr int kRouteTokensPerBlock = 128;
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Route workspace: status word (256 bytes), arrival counter (256 bytes),
+// block histograms [ceil(T/128), E] i32, pair ranks [T*k] i32.  Returns the
+// total size.
+inline size_t route_ws_layout(int64_t T, int E, int k, size_t* off_arr, size_t* off_hist, size_t* off_rank)
+{
+    const int64_t nblocks = ceil_div64(T > 0 ? T : 1, kRouteTokensPerBlock);
+    size_t o = 256;
+    *off_arr = o;
+    o += 256;
+    *off_hist = o;
+    o = align_up(o + static_cast<size_t>(nblocks) * (E > 0 ? E : 1) * 4, 256);
+    *off_rank = o;
+    o = align_up(o + static_cast<size_t>(T > 0 ? T : 1) * (k > 0 ? k : 1) * 4, 256);
+    return o;
+}
 
 // Records a caller's timing event on s.  Inside a stream capture a plain
 // record only orders the capture; the external flag makes it an event node
@@ -32,7 +49,6 @@ inline cudaError_t record_event(void* ev, cudaStream_t s)
                ? cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), s, cudaEventRecordExternal)
                : cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
 }
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct DeviceInfo {
     int sm_count;
@@ -62,6 +78,15 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
 
 cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
                            float* out, uint16_t* out_bf16, int* status, cudaStream_t s);
+// Combine through a row map: out[t] = rs * sum_j y[rows[t*k + j]] over the
+// slots whose row is >= 0, in slot order; rows >= y_nrows set a status bit.
+cudaError_t launch_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int k,
+                                float rs, float* out, uint16_t* out_bf16, int* status, cudaStream_t s);
+
+// The stable permutation of pairs by key (A2 on caller-given ids): block
+// ranks, expert scan, scatter (route_rank_kernel, route_scatter_kernel).
+cudaError_t launch_permute(const int32_t* ids, int64_t T, int E, int k, int32_t* offsets, int32_t* sorted_pairs,
+                           int32_t* block_hist, int32_t* local_rank, int* arrivals, cudaStream_t s);
 
 struct FfnArgs {
     const uint8_t* codes;
@@ -82,6 +107,8 @@ struct FfnArgs {
     const uint8_t* w_down;
     const float* s_down;
     float* y;
+    const int32_t* y_rows;  // nullable: y row of each pair (-1: pair not written)
+    int64_t y_nrows;        // rows of y when y_rows is given
     // workspace pieces
     int* status;
     uint8_t* a_sorted;   // [P, H]

@@ -292,6 +292,32 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
     return cudaGetLastError();
 }
 
+cudaError_t launch_permute(const int32_t* ids, int64_t T, int E, int k, int32_t* offsets, int32_t* sorted_pairs,
+                           int32_t* block_hist, int32_t* local_rank, int* arrivals, cudaStream_t s)
+{
+    if (T == 0 || k == 0) {
+        zero_offsets_kernel<<<1, 256, 0, s>>>(offsets, E + 1);
+        return cudaGetLastError();
+    }
+    // the rank kernel's arrival counter starts at zero (route_topk resets it
+    // on the routing path)
+    cudaError_t err = cudaMemsetAsync(arrivals, 0, sizeof(int), s);
+    if (err != cudaSuccess) return err;
+    const int nblocks = static_cast<int>(ceil_div64(T, kRouteTokensPerBlock));
+    const size_t smem = rank_smem(E);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(route_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+    }
+    route_rank_kernel<<<nblocks, kRankThreads, smem, s>>>(ids, T, E, k, block_hist, local_rank, arrivals, offsets);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int64_t P = T * k;
+    route_scatter_kernel<<<static_cast<int>(ceil_div64(P, 256)), 256, 0, s>>>(ids, P, k, E, block_hist, local_rank,
+                                                                             offsets, sorted_pairs);
+    return cudaGetLastError();
+}
+
 }  // namespace fp8moe
 
 // ---------------------------------------------------------------------------

@@ -281,6 +281,59 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Expert parallelism across `world` GPUs ("next" row of the plan; reading:
+ * the layer shards by expert with one exchange on each side, and each
+ * token's k slot rows are summed on its home GPU in slot order, so a row's
+ * bits do not depend on the sharding -- "GLM-5.3-Flash EXL3 on CUDA ...",
+ * exactness note).  Rank r owns experts [r*E/world, (r+1)*E/world) and is
+ * home to tokens [r*T_home, (r+1)*T_home).  Every rank routes all T tokens.
+ *
+ * moe_ep_plan: from the replicated topk_ids [T, top_k] (read):
+ *   local_ids  [T, top_k] int32: the rank's own experts renumbered from 0,
+ *              -1 for the others (input of moe_permute / the grouped FFN);
+ *   send_rows  [T*top_k]  int32: row of each own pair in the rank's send
+ *              buffer (-1: not own), grouped by home rank, pair order inside
+ *              each group (y_rows of moe_grouped_ffn_rows);
+ *   recv_rows  [T_home, top_k] int32: row of each home slot in the receive
+ *              buffer, grouped by owner rank in rank order (-1: empty slot;
+ *              moe_combine_rows);
+ *   offs_oh, offs_ho  [world*world + 1] int32: exclusive prefixes of the
+ *              pair counts by (owner, home) and by (home, owner); rank r
+ *              sends offs_oh[r*w+h+1] - offs_oh[r*w+h] rows to home h and
+ *              receives offs_ho[r*w+o+1] - offs_ho[r*w+o] rows from owner o.
+ * Both sides take rows in pair order, so no indices travel with them.
+ * Limits: E % world == 0, world*world <= 1024, T_home*world >= T; workspace
+ * moe_ep_plan_workspace_bytes(T, top_k, world).
+ *
+ * moe_permute: the stable permutation of moe_route (A2) on caller-given ids
+ * (ids outside [0, E) are skipped); workspace moe_route_workspace_bytes.
+ *
+ * moe_grouped_ffn_rows: moe_grouped_ffn whose down epilogue writes pair p
+ * to row y_rows[p] of y (y_nrows rows; -1: not written; a row >= y_nrows is
+ * a device fault, MOE_DEV_BAD_PAIR).  y_rows == NULL is moe_grouped_ffn.
+ *
+ * moe_combine_rows: out[t] = routed_scaling * sum over j in slot order of
+ * y[rows[t*top_k + j]] for rows >= 0 (rows >= y_nrows: MOE_DEV_BAD_PAIR);
+ * ws as moe_combine.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ep_plan_workspace_bytes(int64_t T, int top_k, int world);
+MOE_API int moe_ep_plan(const int32_t* topk_ids, int64_t T, int top_k, int E, int world, int rank, int64_t T_home,
+                        int32_t* local_ids, int32_t* send_rows, int32_t* recv_rows, int32_t* offs_oh,
+                        int32_t* offs_ho, void* ws, size_t ws_bytes, void* stream);
+MOE_API int moe_permute(const int32_t* ids, int64_t T, int E, int top_k, int32_t* expert_offsets,
+                        int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream);
+MOE_API int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t T, int H,
+                                 const int32_t* topk_ids, const float* topk_w, int top_k,
+                                 const int32_t* expert_offsets, const int32_t* sorted_pairs, int E, int I,
+                                 const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up, const float* s_up,
+                                 const uint8_t* w_down, const float* s_down, float* y, const int32_t* y_rows,
+                                 int64_t y_nrows, void* ws, size_t ws_bytes, void* stream,
+                                 void* const* stage_events);
+MOE_API int moe_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int top_k,
+                             float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_layer -- the whole routed-expert layer in one call: moe_route_quant,
  * moe_grouped_ffn and moe_combine, stream-ordered, over one caller
  * workspace that also holds the intermediates (codes, scales, routing,

@@ -57,3 +57,41 @@ def test_single_rank_no_process_group():
     w, r, _ = bench.dist_setup("gloo")
     assert (w, r) == (1, 0)
     assert bench.max_over_ranks(1, 3.5, device="cpu") == 3.5
+
+
+# ---- the expert-parallel row exchange (point-to-point; gloo on CPU here,
+# ---- NCCL over NVLink on GPUs)
+
+_COUNTS = [[2, 0, 3], [1, 4, 0], [0, 2, 5]]  # rows rank src sends to rank dst
+
+
+def _exchange_worker(rank, world, port, out):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    bench.dist_setup("gloo")
+    from fp8_blockwise_routed_b200 import ep
+    send_counts = _COUNTS[rank]
+    recv_counts = [_COUNTS[src][rank] for src in range(world)]
+    H = 4
+    rows = []
+    for dst in range(world):
+        for i in range(send_counts[dst]):
+            rows.append([rank * 1000 + dst * 100 + i + 0.25 * c for c in range(H)])
+    send = torch.tensor(rows, dtype=torch.float32) if rows else torch.zeros((0, H))
+    recv = torch.full((sum(recv_counts), H), -1.0)
+    ep.exchange_rows(send, send_counts, recv, recv_counts)
+    bench.barrier(world)
+    torch.distributed.destroy_process_group()
+    out[rank] = recv.tolist()
+
+
+def test_expert_parallel_row_exchange_three_gloo_ranks():
+    world = 3
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_exchange_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    for dst in range(world):
+        want = [[src * 1000 + dst * 100 + i + 0.25 * c for c in range(4)]
+                for src in range(world) for i in range(_COUNTS[src][dst])]
+        assert out[dst] == want
