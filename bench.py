@@ -17,8 +17,11 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
                 copy bandwidth;
   cpu_baseline  the oracle (plain C, FP64) timed on a bounded token sample
                 on this host's cores;
-  e2e           the same metric with host buffers: pinned H2D of x and
-                logits, the three calls, D2H of the FP32 output, per step;
+  e2e           the same metric with host buffers: every step copies its
+                x and logits from pinned host memory and its FP32 output
+                back, pipelined over two layer plans (copy-in, compute and
+                copy-out streams overlap); e2e_serial does the same one step
+                after the other;
   stages        per-launch-group milliseconds from CUDA events;
   clocks        nvidia-smi samples taken during the timed region.
 """
@@ -255,6 +258,52 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+class E2EPipeline:
+    """Host -> device -> host loop over layer plans with double-buffered
+    inputs: a copy-in stream, the compute stream and a copy-out stream,
+    ordered by events so that a plan's inputs are overwritten only after its
+    previous launch has read them and its output only after it was copied
+    out."""
+
+    def __init__(self, plans, x_ins, lg_ins, x_h, lg_h, out_hs):
+        self.plans, self.x_ins, self.lg_ins = plans, x_ins, lg_ins
+        self.x_h, self.lg_h, self.out_hs = x_h, lg_h, out_hs
+        self.h2d, self.comp, self.d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        n = len(plans)
+        self.ev_in = [torch.cuda.Event() for _ in range(n)]
+        self.ev_comp = [torch.cuda.Event() for _ in range(n)]
+        self.ev_out = [torch.cuda.Event() for _ in range(n)]
+
+    def run(self, steps: int) -> float:
+        """Runs `steps` steps; returns their device time in ms (first copy in
+        to last copy out)."""
+        n = len(self.plans)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(self.h2d)
+        for i in range(steps):
+            b = i % n
+            used = i >= n
+            if used:
+                self.h2d.wait_event(self.ev_comp[b])  # plan b has read its previous inputs
+            with torch.cuda.stream(self.h2d):
+                self.x_ins[b].copy_(self.x_h, non_blocking=True)
+                self.lg_ins[b].copy_(self.lg_h, non_blocking=True)
+                self.ev_in[b].record(self.h2d)
+            self.comp.wait_event(self.ev_in[b])
+            if used:
+                self.comp.wait_event(self.ev_out[b])  # its previous output has been copied out
+            self.plans[b].launch(self.comp)
+            self.ev_comp[b].record(self.comp)
+            self.d2h.wait_event(self.ev_comp[b])
+            with torch.cuda.stream(self.d2h):
+                self.out_hs[b].copy_(self.plans[b].out, non_blocking=True)
+                self.ev_out[b].record(self.d2h)
+        t1.record(self.d2h)
+        t1.synchronize()
+        return t0.elapsed_time(t1)
+
+
 def workload_config(wl):
     return {"workload": f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} top_k={wl.k} I={wl.I} "
                         f"rs={wl.routed_scaling} x={wl.x_dist} logits={wl.logit_dist}",
@@ -388,7 +437,23 @@ def main():
     e1.record(s)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+    e2e_serial_ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+
+    # The same, pipelined as a serving loop runs it: two plans over
+    # double-buffered inputs; step i+1's inputs are copied in while step i
+    # computes and step i-1's output is copied out (three streams, ordered
+    # by events).  Every step still copies its own inputs and result.
+    x_in2 = torch.empty_like(d["x"])
+    lg_in2 = torch.empty_like(d["logits"])
+    plan2 = fm.LayerPlan(x_in2, lg_in2, wl.k, d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"],
+                         d["s_down"], wl.routed_scaling)
+    out_h2 = torch.empty_like(out_h).pin_memory()
+    pipe = E2EPipeline([plan, plan2], [x_in, x_in2], [lg_in, lg_in2], x_h, lg_h, [out_h, out_h2])
+    pipe.run(2)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, pipe.run(args.steps)) / args.steps
+    status |= plan2.device_status()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -420,7 +485,10 @@ def main():
             "stages_ms": stage_ms,
             "stages_ms_last_timed_step": last_ms,
             "ms_per_step_three_calls": ms_calls,
+            "e2e_serial": {"value": whole_job_tokens_per_s(world, wl.T, e2e_serial_ms), "unit": "tokens/s",
+                           "ms_per_step": e2e_serial_ms},
             "e2e": {"value": whole_job_tokens_per_s(world, wl.T, e2e_ms), "unit": "tokens/s",
+                    "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i's compute",
                     "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                     "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms},
             "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
@@ -434,6 +502,7 @@ def main():
             line["clocks"] = clocks
         print(json.dumps(line), flush=True)
     plan.close()
+    plan2.close()
     if world > 1:
         torch.distributed.destroy_process_group()
 
