@@ -230,7 +230,13 @@ def run_reference(args, wl):
         return
     import oracle
 
-    d = mi.make_inputs(wl, 0, "cpu")
+    # the same seeded inputs as the GPU arm when a GPU is present (drawn
+    # there in seconds, then copied to the host); only the oracle's
+    # evaluation on the host cores is timed
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = {key: v.cpu() for key, v in mi.make_inputs(wl, rank_seed(0), gen_dev).items()}
+    if gen_dev == "cuda":
+        torch.cuda.empty_cache()
     n = 32  # tokens per step: about a third of a second of oracle work on 16 cores
     W = [d[k] for k in ("w_gate", "s_gate", "w_up", "s_up", "w_down", "s_down")]
     oracle.build()
