@@ -233,6 +233,38 @@ def moe_ffn(codes, act_scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_dow
     return res
 
 
+def route_shared(logits, top_k: int):
+    """Routing with the shared expert as one more slot after the top-k
+    ("GLM-5.3-Flash EXL3 on CUDA ...": all nine slots planned with E+1 expert
+    ids, the shared id skipped by the routed kernels).  Reading: the extra
+    slot k holds id E with weight 1 (the shared expert is not gated)."""
+    ids, w = route(logits, top_k)
+    T = ids.shape[0]
+    E = int(logits.shape[1])
+    ids2 = np.concatenate([ids, np.full((T, 1), E, np.int32)], axis=1)
+    w2 = np.concatenate([w, np.ones((T, 1), w.dtype)], axis=1)
+    return ids2, w2
+
+
+def moe_layer_shared(x_bf16, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down,
+                     routed_scaling, shared_rows, tokens=None):
+    """The layer with a shared-expert slot: the routed experts as in
+    moe_layer, plus the caller's shared-expert row for each token, added
+    unscaled: out[t] = routed_scaling * sum_j w_j o_j + shared[t] (the
+    routed scaling applies to the routed experts only, as in the pages'
+    layer, where routed scaling and the shared experts are separate parts).
+    shared_rows: [T, H] (float32 or float64), the rows the caller writes into
+    the shared slot."""
+    res = moe_layer(x_bf16, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling,
+                    tokens=tokens)
+    sh = np.asarray(shared_rows.detach().cpu().numpy() if hasattr(shared_rows, "detach") else shared_rows,
+                    dtype=np.float64)
+    if tokens is not None:
+        sh = sh[np.asarray(tokens)]
+    res["out"] = res["out"] + sh
+    return res
+
+
 def moe_layer(x_bf16, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down,
               routed_scaling, tokens=None, **kw):
     """The whole path in the pages' order: quantise activations, route,
