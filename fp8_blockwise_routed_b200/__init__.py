@@ -85,6 +85,10 @@ def lib() -> ctypes.CDLL:
                                            P, sz, P, P]
         L.moe_combine_rows.restype = i32
         L.moe_combine_rows.argtypes = [P, i64, P, i64, i32, i32, ctypes.c_float, P, P, P, sz, P]
+        L.moe_route_shared.restype = i32
+        L.moe_route_shared.argtypes = [P, i64, i32, i32, P, P, P, P, P, sz, P]
+        L.moe_combine_shared.restype = i32
+        L.moe_combine_shared.argtypes = [P, P, i64, i32, i32, i32, ctypes.c_float, P, P, P, sz, P]
         L.moe_route_quant.restype = i32
         L.moe_route_quant.argtypes = [P, P, i64, i32, i32, i32, P, P, P, P, P, P, P, sz, P]
         L.moe_ffn_workspace_bytes.restype = sz
@@ -298,6 +302,24 @@ class LayerPlan:
             self.close()
         except Exception:
             pass
+
+
+def moe_route_shared(logits, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, stream=None):
+    """moe_route plus the shared-expert slot: topk_ids / topk_w [T, top_k+1]
+    with slot top_k = (E, 1.0); sorted_pairs [T*(top_k+1)] (routed pairs)."""
+    T, E = logits.shape
+    _check(lib().moe_route_shared(_p(logits), T, E, top_k, _p(topk_ids), _p(topk_w), _p(expert_offsets),
+                                  _p(sorted_pairs), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "moe_route_shared")
+
+
+def moe_combine_shared(y, topk_ids, num_experts, routed_scaling, out_f32, out_bf16, ws, stream=None):
+    """moe_combine with the shared-expert slot (id num_experts) added after
+    the routed scaling."""
+    T, k, H = y.shape
+    _check(lib().moe_combine_shared(_p(y), _p(topk_ids), T, H, k, num_experts, routed_scaling, _p(out_f32),
+                                    _p(out_bf16), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "moe_combine_shared")
 
 
 def moe_ep_plan_workspace_bytes(T: int, top_k: int, world: int) -> int:

@@ -122,25 +122,27 @@ namespace {
 
 int route_common(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
                  int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream,
-                 const fp8moe::QuantArgs* quant, const char* what)
+                 const fp8moe::QuantArgs* quant, const char* what, int shared = 0)
 {
-    if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 0 || top_k > E || top_k > MOE_MAX_TOP_K)
+    if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 0 || top_k > E || top_k + shared > MOE_MAX_TOP_K)
         return MOE_ERR_INVALID_ARG;
-    if (T > (int64_t(1) << 31) / (top_k > 0 ? top_k : 1) - 1) return MOE_ERR_UNSUPPORTED;
+    if (shared && top_k < 1) return MOE_ERR_INVALID_ARG;
+    const int kp = top_k + shared;
+    if (T > (int64_t(1) << 31) / (kp > 0 ? kp : 1) - 1) return MOE_ERR_UNSUPPORTED;
     if (!expert_offsets || !ws) return MOE_ERR_INVALID_ARG;
     if (T > 0 && top_k > 0 && (!logits || !topk_ids || !topk_w || !sorted_pairs)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(logits) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) ||
         !aligned16(sorted_pairs) || !aligned16(ws))
         return MOE_ERR_ALIGNMENT;
     size_t off_arr, off_hist, off_rank;
-    if (ws_bytes < route_layout(T, E, top_k, &off_arr, &off_hist, &off_rank)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < route_layout(T, E, kp, &off_arr, &off_hist, &off_rank)) return MOE_ERR_WORKSPACE;
     if (int r = check_device()) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (int r = clear_status(ws, s)) return r;
     uint8_t* w8 = static_cast<uint8_t*>(ws);
     cudaError_t err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
                                    reinterpret_cast<int32_t*>(w8 + off_hist), reinterpret_cast<int32_t*>(w8 + off_rank),
-                                   reinterpret_cast<int*>(w8 + off_arr), quant, s);
+                                   reinterpret_cast<int*>(w8 + off_arr), quant, s, shared);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, what);
 }
 
@@ -151,6 +153,13 @@ int moe_route(const float* logits, int64_t T, int E, int top_k, int32_t* topk_id
 {
     return route_common(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, ws_bytes, stream,
                         nullptr, "moe_route");
+}
+
+int moe_route_shared(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
+                     int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes, void* stream)
+{
+    return route_common(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, ws_bytes, stream,
+                        nullptr, "moe_route_shared", 1);
 }
 
 int moe_route_quant(const float* logits, const uint16_t* x, int64_t T, int H, int E, int top_k, int32_t* topk_ids,
@@ -272,6 +281,24 @@ int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int H, int t
     cudaError_t err = launch_combine(y, topk_ids, T, H, top_k, E, routed_scaling, out_f32, out_bf16,
                                      static_cast<int*>(ws), s);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
+}
+
+int moe_combine_shared(const float* y, const int32_t* topk_ids, int64_t T, int H, int top_k, int E,
+                       float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                       void* stream)
+{
+    if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (top_k < 1 || top_k > MOE_MAX_TOP_K || E < 1 || E > MOE_MAX_EXPERTS) return MOE_ERR_INVALID_ARG;
+    if (!ws || (T > 0 && (!out_f32 || !y || !topk_ids))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(topk_ids) || !aligned16(out_f32) || !aligned16(out_bf16) || !aligned16(ws))
+        return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    if (int r = check_device()) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int r = clear_status(ws, s)) return r;
+    cudaError_t err = launch_combine(y, topk_ids, T, H, top_k, E, routed_scaling, out_f32, out_bf16,
+                                     static_cast<int*>(ws), s, E);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine_shared");
 }
 
 int moe_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int top_k,

@@ -1,5 +1,6 @@
 // combine.cu -- out[t,:] = routed_scaling * sum_j y[t,j,:] over valid slots,
-// in slot order, FP32 ("Full GLM-5.3 streamed FP8 GPU prefill ...",
+// in slot order, FP32 (plus, with a shared-expert slot, that slot's row added
+// after the scaling) ("Full GLM-5.3 streamed FP8 GPU prefill ...",
 // "Design": routed scaling kept with the routed-expert sum; "GLM-5.3-Flash
 // EXL3 on CUDA ...", commit text: routed FP32 rows).
 //
@@ -36,7 +37,7 @@ constexpr int kSlotBatch = 8;  // slot rows loaded together per thread
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ ids,
                                                       int64_t T, int H4, int k, int E, float rs,
                                                       float4* __restrict__ out, uint2* __restrict__ out_bf16,
-                                                      int* __restrict__ status)
+                                                      int* __restrict__ status, int shared_id)
 {
     const int64_t n = T * H4;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -44,6 +45,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
         const int64_t t = i / H4;
         const int64_t c = i - t * H4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 sh = make_float4(0.f, 0.f, 0.f, 0.f);
+        bool any_shared = false;
         // slots in batches: the batch's loads are all issued before the sums,
         // which then run in slot order over the valid slots only
         for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
@@ -53,9 +56,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
             for (int u = 0; u < kSlotBatch; ++u) {
                 const int j = j0 + u;
                 const int e = (j < k) ? __ldg(ids + t * k + j) : -1;
-                if ((e < -1 || e >= E) && c == 0) atomicOr(status, kDevBadExpertId);
-                ok[u] = e >= 0 && e < E;
+                const bool is_sh = shared_id >= 0 && e == shared_id;
+                if ((e < -1 || e >= E) && !is_sh && c == 0) atomicOr(status, kDevBadExpertId);
+                ok[u] = (e >= 0 && e < E) || is_sh;
                 v[u] = ok[u] ? ld_stream_f4(y + (t * k + j) * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (is_sh) {  // the shared expert's row: summed apart, not scaled
+                    ok[u] = false;
+                    any_shared = true;
+                    sh.x += v[u].x;
+                    sh.y += v[u].y;
+                    sh.z += v[u].z;
+                    sh.w += v[u].w;
+                }
             }
 #pragma unroll
             for (int u = 0; u < kSlotBatch; ++u) {
@@ -66,7 +78,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
                 acc.w += v[u].w;
             }
         }
-        const float4 o = make_float4(rs * acc.x, rs * acc.y, rs * acc.z, rs * acc.w);
+        float4 o = make_float4(rs * acc.x, rs * acc.y, rs * acc.z, rs * acc.w);
+        if (any_shared) o = make_float4(o.x + sh.x, o.y + sh.y, o.z + sh.z, o.w + sh.w);
         out[i] = o;
         if (out_bf16) out_bf16[i] = make_uint2(bf16x2_rn(o.x, o.y), bf16x2_rn(o.z, o.w));
     }
@@ -130,7 +143,7 @@ cudaError_t launch_combine_rows(const float* y, int64_t y_nrows, const int32_t* 
 }
 
 cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
-                           float* out, uint16_t* out_bf16, int* status, cudaStream_t s)
+                           float* out, uint16_t* out_bf16, int* status, cudaStream_t s, int shared_id)
 {
     const int H4 = H / 4;
     const int64_t n = T * H4;
@@ -141,7 +154,8 @@ cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H,
     const int64_t cap = static_cast<int64_t>(di.sm_count) * 8 * 8;
     const int grid = static_cast<int>(want < cap ? want : cap);
     combine_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), ids, T, H4, k, E, rs,
-                                        reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16), status);
+                                        reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16), status,
+                                        shared_id);
     return cudaGetLastError();
 }
 

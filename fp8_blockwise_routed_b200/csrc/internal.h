@@ -70,14 +70,18 @@ struct QuantArgs {
     float* scales;      // [T, H/128]
 };
 
-// block_hist: [ceil(T/128), E] i32; local_rank: [T*k] i32; arrivals: one int
-// (reset by the first launch, counted by the second).  quant may be null.
+// block_hist: [ceil(T/128), E] i32; local_rank: [T*(k+shared)] i32;
+// arrivals: one int (reset by the first launch, counted by the second).
+// quant may be null.  shared = 1 appends the shared-expert slot (id E,
+// weight 1) after the top-k: ids and w are then [T, k+1].
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w,
                          int32_t* offsets, int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank,
-                         int* arrivals, const QuantArgs* quant, cudaStream_t s);
+                         int* arrivals, const QuantArgs* quant, cudaStream_t s, int shared = 0);
 
+// shared_id >= 0: slots with that id are the shared expert's rows, summed
+// apart and added after the routed scaling.
 cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H, int k, int E, float rs,
-                           float* out, uint16_t* out_bf16, int* status, cudaStream_t s);
+                           float* out, uint16_t* out_bf16, int* status, cudaStream_t s, int shared_id = -1);
 // Combine through a row map: out[t] = rs * sum_j y[rows[t*k + j]] over the
 // slots whose row is >= 0, in slot order; rows >= y_nrows set a status bit.
 cudaError_t launch_combine_rows(const float* y, int64_t y_nrows, const int32_t* rows, int64_t T, int H, int k,

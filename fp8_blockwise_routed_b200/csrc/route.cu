@@ -102,7 +102,8 @@ __device__ __forceinline__ void topk_token(const float* __restrict__ row, int E,
 // arrival counter (this launch precedes it in stream order).
 template <int VPL>
 __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float* __restrict__ logits, int64_t T,
-                                                                     int E, int k, int32_t* __restrict__ ids,
+                                                                     int E, int k, int shared,
+                                                                     int32_t* __restrict__ ids,
                                                                      float* __restrict__ w, int* __restrict__ arrivals,
                                                                      int64_t n_topk, const uint4* __restrict__ qx,
                                                                      int64_t q_groups, uint8_t* __restrict__ q_codes,
@@ -116,7 +117,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32) route_topk_kernel(const float
     const int lane = threadIdx.x & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5);
     if (t >= T) return;
-    topk_token<VPL>(logits + t * E, E, k, ids + t * k, w + t * k, lane);
+    const int kout = k + shared;  // the shared-expert slot, if any, follows the top-k
+    topk_token<VPL>(logits + t * E, E, k, ids + t * kout, w + t * kout, lane);
+    if (shared && lane == 0) {
+        ids[t * kout + k] = E;
+        w[t * kout + k] = 1.0f;
+    }
 }
 
 // One block per kRouteTokensPerBlock tokens; pairs of the block are taken
@@ -242,7 +248,7 @@ size_t rank_smem(int E) { return (33ull * E) * sizeof(int32_t); }
 
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* offsets,
                          int32_t* sorted_pairs, int32_t* block_hist, int32_t* local_rank, int* arrivals,
-                         const QuantArgs* quant, cudaStream_t s)
+                         const QuantArgs* quant, cudaStream_t s, int shared)
 {
     int64_t q_groups = 0, q_blocks = 0;
     DeviceInfo di;
@@ -257,7 +263,7 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
         if (err != cudaSuccess || q_blocks == 0) return err;
         // top_k == 0 or T == 0: nothing is routed; ids/w/sorted_pairs are empty
         route_topk_kernel<2><<<static_cast<int>(q_blocks), kTopkWarps * 32, 0, s>>>(
-            logits, 0, E, k, ids, w, arrivals, 0, reinterpret_cast<const uint4*>(quant->x), q_groups, quant->codes,
+            logits, 0, E, k, 0, ids, w, arrivals, 0, reinterpret_cast<const uint4*>(quant->x), q_groups, quant->codes,
             quant->scales);
         return cudaGetLastError();
     }
@@ -267,13 +273,13 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
     uint8_t* qc = quant ? quant->codes : nullptr;
     float* qs = quant ? quant->scales : nullptr;
     if (E <= 64)
-        route_topk_kernel<2><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+        route_topk_kernel<2><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, shared, ids, w, arrivals, n_topk, qx,
                                                                q_groups, qc, qs);
     else if (E <= 256)
-        route_topk_kernel<8><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+        route_topk_kernel<8><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, shared, ids, w, arrivals, n_topk, qx,
                                                                q_groups, qc, qs);
     else
-        route_topk_kernel<32><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, ids, w, arrivals, n_topk, qx,
+        route_topk_kernel<32><<<grid, kTopkWarps * 32, 0, s>>>(logits, T, E, k, shared, ids, w, arrivals, n_topk, qx,
                                                                 q_groups, qc, qs);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
@@ -284,10 +290,12 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                                    static_cast<int>(smem));
         if (err != cudaSuccess) return err;
     }
-    route_rank_kernel<<<nblocks, kRankThreads, smem, s>>>(ids, T, E, k, block_hist, local_rank, arrivals, offsets);
+    // the pairs include the shared slot (id E), which the ranking skips
+    const int kp = k + shared;
+    route_rank_kernel<<<nblocks, kRankThreads, smem, s>>>(ids, T, E, kp, block_hist, local_rank, arrivals, offsets);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const int64_t P = T * k;
-    route_scatter_kernel<<<static_cast<int>(ceil_div64(P, 256)), 256, 0, s>>>(ids, P, k, E, block_hist, local_rank,
+    const int64_t P = T * kp;
+    route_scatter_kernel<<<static_cast<int>(ceil_div64(P, 256)), 256, 0, s>>>(ids, P, kp, E, block_hist, local_rank,
                                                                              offsets, sorted_pairs);
     return cudaGetLastError();
 }
@@ -405,7 +413,7 @@ extern "C" int moe_route_noalloc(const float* logits, int64_t T, int E, int top_
     // counter, histograms and ranks it later reads.
     err = launch_route(logits, T, E, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs,
                        reinterpret_cast<int32_t*>(base + off_hist), reinterpret_cast<int32_t*>(base + off_rank),
-                       reinterpret_cast<int*>(base), nullptr, static_cast<cudaStream_t>(stream));
+                       reinterpret_cast<int*>(base), nullptr, static_cast<cudaStream_t>(stream), 0);
     if (err != cudaSuccess) {
         std::snprintf(g_noalloc_error, sizeof(g_noalloc_error), "launch: %s", cudaGetErrorString(err));
         return MOE_ERR_CUDA;

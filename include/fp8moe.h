@@ -281,6 +281,33 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Shared-expert slot.  The pages plan a shared expert as one more slot after
+ * the routed ones ("GLM-5.3-Flash EXL3 on CUDA ...": all nine slots planned
+ * with E+1 expert ids, the shared id skipped before any routed payload is
+ * read, routed FP32 rows written in place).  Readings: the shared slot is
+ * slot top_k, id E, weight 1; the caller computes the shared expert and
+ * writes its row into that slot of y; the combine adds it after the routed
+ * scaling, out = routed_scaling * sum(routed slots) + shared (the pages keep
+ * routed scaling and the shared experts as separate parts of the layer).
+ *
+ * moe_route_shared: moe_route whose topk_ids / topk_w are [T, top_k+1] with
+ *   slot top_k = (E, 1.0) and whose sorted_pairs is [T*(top_k+1)]; the
+ *   permutation holds the routed pairs only (the shared id is skipped), so
+ *   moe_grouped_ffn with top_k+1 slots computes the routed rows and leaves the
+ *   shared slot's rows of y untouched.  Workspace:
+ *   moe_route_workspace_bytes(T, E, top_k+1).  1 <= top_k <= 31.
+ * moe_combine_shared: moe_combine over top_k slots (the shared one
+ *   included) in which the slots holding id E are summed apart (slot order)
+ *   and added to routed_scaling * (sum of the routed slots).
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_route_shared(const float* logits, int64_t T, int E, int top_k, int32_t* topk_ids, float* topk_w,
+                             int32_t* expert_offsets, int32_t* sorted_pairs, void* ws, size_t ws_bytes,
+                             void* stream);
+MOE_API int moe_combine_shared(const float* y, const int32_t* topk_ids, int64_t T, int H, int top_k, int E,
+                               float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* ---------------------------------------------------------------------------
  * Expert parallelism across `world` GPUs ("next" row of the plan; reading:
  * the layer shards by expert with one exchange on each side, and each
  * token's k slot rows are summed on its home GPU in slot order, so a row's
