@@ -34,6 +34,9 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi)
 
 constexpr int kSlotBatch = 8;  // slot rows loaded together per thread
 
+// SHARED: slots holding shared_id are the shared expert's rows, summed apart
+// and added after the routed scaling (moe_combine_shared).
+template <bool SHARED>
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ ids,
                                                       int64_t T, int H4, int k, int E, float rs,
                                                       float4* __restrict__ out, uint2* __restrict__ out_bf16,
@@ -51,27 +54,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
         // which then run in slot order over the valid slots only
         for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
             float4 v[kSlotBatch];
-            bool ok[kSlotBatch];
+            bool ok[kSlotBatch], shr[kSlotBatch];
 #pragma unroll
             for (int u = 0; u < kSlotBatch; ++u) {
                 const int j = j0 + u;
                 const int e = (j < k) ? __ldg(ids + t * k + j) : -1;
-                const bool is_sh = shared_id >= 0 && e == shared_id;
-                if ((e < -1 || e >= E) && !is_sh && c == 0) atomicOr(status, kDevBadExpertId);
-                ok[u] = (e >= 0 && e < E) || is_sh;
+                shr[u] = SHARED && e == shared_id;
+                if ((e < -1 || e >= E) && !shr[u] && c == 0) atomicOr(status, kDevBadExpertId);
+                ok[u] = (e >= 0 && e < E) || shr[u];
                 v[u] = ok[u] ? ld_stream_f4(y + (t * k + j) * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-                if (is_sh) {  // the shared expert's row: summed apart, not scaled
-                    ok[u] = false;
+            }
+#pragma unroll
+            for (int u = 0; u < kSlotBatch; ++u) {
+                if (!ok[u]) continue;
+                if (SHARED && shr[u]) {  // the shared expert's row: summed apart, not scaled
                     any_shared = true;
                     sh.x += v[u].x;
                     sh.y += v[u].y;
                     sh.z += v[u].z;
                     sh.w += v[u].w;
+                    continue;
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < kSlotBatch; ++u) {
-                if (!ok[u]) continue;
                 acc.x += v[u].x;
                 acc.y += v[u].y;
                 acc.z += v[u].z;
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
             }
         }
         float4 o = make_float4(rs * acc.x, rs * acc.y, rs * acc.z, rs * acc.w);
-        if (any_shared) o = make_float4(o.x + sh.x, o.y + sh.y, o.z + sh.z, o.w + sh.w);
+        if (SHARED && any_shared) o = make_float4(o.x + sh.x, o.y + sh.y, o.z + sh.z, o.w + sh.w);
         out[i] = o;
         if (out_bf16) out_bf16[i] = make_uint2(bf16x2_rn(o.x, o.y), bf16x2_rn(o.z, o.w));
     }
@@ -153,9 +156,14 @@ cudaError_t launch_combine(const float* y, const int32_t* ids, int64_t T, int H,
     const int64_t want = ceil_div64(n, 256);
     const int64_t cap = static_cast<int64_t>(di.sm_count) * 8 * 8;
     const int grid = static_cast<int>(want < cap ? want : cap);
-    combine_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), ids, T, H4, k, E, rs,
-                                        reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16), status,
-                                        shared_id);
+    if (shared_id >= 0)
+        combine_kernel<true><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), ids, T, H4, k, E, rs,
+                                                  reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16),
+                                                  status, shared_id);
+    else
+        combine_kernel<false><<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), ids, T, H4, k, E, rs,
+                                                   reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16),
+                                                   status, -1);
     return cudaGetLastError();
 }
 
