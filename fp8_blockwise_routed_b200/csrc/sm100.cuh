@@ -167,28 +167,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, fl
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-// L2 prefetch of the cache line holding a global address.
-__device__ __forceinline__ void prefetch_l2(const void* ptr)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-// L2 prefetch of a tile (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int c0, int c1)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tmap(const void* tmap)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -241,29 +219,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
                  : "memory");
 }
 
-// 32 consecutive FP32 columns of this thread's TMEM lane, loaded and waited
-// for in one statement so that no use of the values can be scheduled
-// before the wait.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Split form: issue a 32-column load into r, and wait for all loads of this
-// thread.  The wait takes r as in/out operands, so the compiler cannot move
+// 32 consecutive FP32 columns of this thread's TMEM lane, in two parts:
+// issue the load into r, then wait for all loads of this thread.  The wait takes r as in/out operands, so the compiler cannot move
 // a use of r above it, while uses of other registers (an earlier load's
 // values) can run between issue and wait.
 __device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32])
