@@ -185,3 +185,41 @@ def test_device_status_bad_offsets():
     assert st & fm.DEV_BAD_OFFSETS
     assert not (st & fm.DEV_WAIT_TIMEOUT)
     assert torch.all(y == 0)
+
+
+def test_exact_integer_layer():
+    """Exact-arithmetic case: every value on the path is an integer the
+    formats hold exactly, so the GPU output must equal an integer matmul bit
+    for bit.  x rows hold 448 (column 0: activation scale exactly 1), 32 and 1
+    (columns 1, 2); weight scales are 1; gate weights give g = 32 for every
+    intermediate column, where SiLU(g) = g in FP32 (e^-32 is below half an
+    ulp of 1); up weights give u = n mod 15, so h = 32 u is a multiple of 32
+    up to 448 (E4M3-exact, and every 128-group's amax is 448: intermediate
+    scale exactly 1); down weights are small integers; each token is routed
+    to one expert (weight 1) and routed_scaling is 1."""
+    T, H, I, E, k = 300, 256, 256, 4, 1
+    dev = "cuda"
+    x = torch.zeros((T, H), dtype=torch.float32)
+    x[:, 0], x[:, 1], x[:, 2] = 448.0, 32.0, 1.0
+    wg = torch.zeros((E, I, H))
+    wg[:, :, 1] = 1.0                      # g_n = 32
+    wu = torch.zeros((E, I, H))
+    wu[:, :, 2] = (torch.arange(I) % 15).float()   # u_n = n mod 15
+    g = torch.Generator().manual_seed(4)
+    wd = torch.randint(-3, 4, (E, H, I), generator=g).float()
+    logits = torch.full((T, E), -5.0)
+    owner = torch.arange(T) % E
+    logits[torch.arange(T), owner] = 5.0
+
+    def codes(w):
+        return w.to(torch.float8_e4m3fn).view(torch.uint8).to(dev)
+
+    ones_gu = torch.ones((E, I // 128, H // 128), device=dev)
+    ones_d = torch.ones((E, H // 128, I // 128), device=dev)
+    layer = fm.RoutedMoE(codes(wg), ones_gu, codes(wu), ones_gu.clone(), codes(wd), ones_d, k, 1.0, T)
+    out = layer.forward(x.to(torch.bfloat16).to(dev), logits.to(dev))
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    h = (32 * (torch.arange(I) % 15)).to(torch.int64)                 # [I]
+    want = torch.stack([wd[owner[t]].to(torch.int64) @ h for t in range(T)])  # [T, H]
+    assert torch.equal(out.cpu(), want.to(torch.float32))
