@@ -85,6 +85,12 @@ def lib() -> ctypes.CDLL:
                                            P, sz, P, P]
         L.moe_combine_rows.restype = i32
         L.moe_combine_rows.argtypes = [P, i64, P, i64, i32, i32, ctypes.c_float, P, P, P, sz, P]
+        L.moe_grouped_ffn_combine.restype = i32
+        L.moe_grouped_ffn_combine.argtypes = [P, P, i64, i32, P, P, i32, P, P, i32, i32, P, P, P, P, P, P, P,
+                                              ctypes.c_float, P, P, P, sz, P, P]
+        L.moe_layer_plan_create_ex.restype = i32
+        L.moe_layer_plan_create_ex.argtypes = [ctypes.POINTER(ctypes.c_void_p), P, P, i64, i32, i32, i32, i32,
+                                               P, P, P, P, P, P, ctypes.c_float, P, P, P, sz, P, i32]
         L.moe_route_shared.restype = i32
         L.moe_route_shared.argtypes = [P, i64, i32, i32, P, P, P, P, P, sz, P]
         L.moe_combine_shared.restype = i32
@@ -261,7 +267,7 @@ class LayerPlan:
     ``logits`` before ``launch``.  The plan owns its workspace."""
 
     def __init__(self, x, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling,
-                 out_bf16=None, stage_events=None):
+                 out_bf16=None, stage_events=None, fused_combine: bool = False):
         T, E = logits.shape
         H = x.shape[1]
         I = w_gate.shape[1]
@@ -280,9 +286,10 @@ class LayerPlan:
                     e.record()
             evs = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
         h = ctypes.c_void_p(0)
-        _check(lib().moe_layer_plan_create(ctypes.byref(h), _p(logits), _p(x), T, H, E, int(top_k), I,
-                                           *[_p(t) for t in self.w], float(routed_scaling), _p(self.out),
-                                           _p(out_bf16), _p(self.ws), self.ws.numel(), evs), "moe_layer_plan_create")
+        _check(lib().moe_layer_plan_create_ex(ctypes.byref(h), _p(logits), _p(x), T, H, E, int(top_k), I,
+                                              *[_p(t) for t in self.w], float(routed_scaling), _p(self.out),
+                                              _p(out_bf16), _p(self.ws), self.ws.numel(), evs,
+                                              1 if fused_combine else 0), "moe_layer_plan_create")
         self._h = h
 
     def launch(self, stream=None) -> torch.Tensor:
@@ -302,6 +309,24 @@ class LayerPlan:
             self.close()
         except Exception:
             pass
+
+
+def moe_grouped_ffn_combine(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs, w_gate, s_gate,
+                            w_up, s_up, w_down, s_down, y, routed_scaling, out_f32, out_bf16, ws, stream=None,
+                            stage_events=None):
+    """moe_grouped_ffn with the combine fused into the down GEMM: writes
+    out_f32 (and out_bf16) as moe_combine would, bit for bit."""
+    T, H = codes.shape
+    k = topk_ids.shape[1]
+    E, I = w_gate.shape[0], w_gate.shape[1]
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * 4)(*[e.cuda_event for e in stage_events])
+    _check(lib().moe_grouped_ffn_combine(_p(codes), _p(act_scales), T, H, _p(topk_ids), _p(topk_w), k,
+                                         _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate),
+                                         _p(w_up), _p(s_up), _p(w_down), _p(s_down), _p(y), routed_scaling,
+                                         _p(out_f32), _p(out_bf16), _p(ws), ws.numel() * ws.element_size(),
+                                         _s(stream), ev), "moe_grouped_ffn_combine")
 
 
 def moe_route_shared(logits, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, ws, stream=None):

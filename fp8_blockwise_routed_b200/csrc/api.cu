@@ -204,14 +204,22 @@ int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64_t T, in
                                 stage_events);
 }
 
-int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t T, int H, const int32_t* topk_ids,
-                         const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs,
-                         int E, int I, const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
-                         const float* s_up, const uint8_t* w_down, const float* s_down, float* y,
-                         const int32_t* y_rows, int64_t y_nrows, void* ws, size_t ws_bytes, void* stream,
-                         void* const* stage_events)
+}  // extern "C"
+
+namespace {
+
+// moe_grouped_ffn and its variants: a row map for y, or the combine fused
+// into the down GEMM (fuse = 1: out = routed_scaling * slot sum).
+int ffn_call(const uint8_t* codes, const float* act_scales, int64_t T, int H, const int32_t* topk_ids,
+             const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs, int E, int I,
+             const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up, const float* s_up,
+             const uint8_t* w_down, const float* s_down, float* y, const int32_t* y_rows, int64_t y_nrows, void* ws,
+             size_t ws_bytes, void* stream, void* const* stage_events, int fuse, float rs, float* out,
+             uint16_t* out_bf16, const char* what)
 {
     if (y_rows && y_nrows < 0) return MOE_ERR_INVALID_ARG;
+    if (fuse && (y_rows || (T > 0 && !out))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(out_bf16)) return MOE_ERR_ALIGNMENT;
     if (!aligned16(y_rows)) return MOE_ERR_ALIGNMENT;
     if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOP_K) return MOE_ERR_INVALID_ARG;
@@ -226,8 +234,9 @@ int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t 
                           w_up, s_up, w_down, s_down, y, ws};
     for (const void* p : ptrs)
         if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
-    size_t off_a, off_sa, off_h, off_sh;
-    if (ws_bytes < ffn_workspace_layout(T, H, I, top_k, &off_a, &off_sa, &off_h, &off_sh)) return MOE_ERR_WORKSPACE;
+    size_t off_a, off_sa, off_h, off_sh, off_cnt, off_nv;
+    if (ws_bytes < ffn_workspace_layout(T, H, I, top_k, &off_a, &off_sa, &off_h, &off_sh, &off_cnt, &off_nv))
+        return MOE_ERR_WORKSPACE;
     if (int r = check_device()) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (int r = clear_status(ws, s)) return r;
@@ -260,8 +269,42 @@ int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t 
     a.h_codes = w8 + off_h;
     a.h_scales = reinterpret_cast<float*>(w8 + off_sh);
     a.stage_events = stage_events;
+    a.fuse = fuse;
+    a.rs = rs;
+    a.out = out;
+    a.out_bf16 = out_bf16;
+    a.cnt = reinterpret_cast<int*>(w8 + off_cnt);
+    a.nvalid = reinterpret_cast<int32_t*>(w8 + off_nv);
     cudaError_t err = launch_grouped_ffn(a, s);
-    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_ffn");
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_grouped_ffn_rows(const uint8_t* codes, const float* act_scales, int64_t T, int H, const int32_t* topk_ids,
+                         const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs,
+                         int E, int I, const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
+                         const float* s_up, const uint8_t* w_down, const float* s_down, float* y,
+                         const int32_t* y_rows, int64_t y_nrows, void* ws, size_t ws_bytes, void* stream,
+                         void* const* stage_events)
+{
+    return ffn_call(codes, act_scales, T, H, topk_ids, topk_w, top_k, expert_offsets, sorted_pairs, E, I, w_gate,
+                    s_gate, w_up, s_up, w_down, s_down, y, y_rows, y_nrows, ws, ws_bytes, stream, stage_events, 0,
+                    0.f, nullptr, nullptr, "moe_grouped_ffn");
+}
+
+int moe_grouped_ffn_combine(const uint8_t* codes, const float* act_scales, int64_t T, int H,
+                            const int32_t* topk_ids, const float* topk_w, int top_k, const int32_t* expert_offsets,
+                            const int32_t* sorted_pairs, int E, int I, const uint8_t* w_gate, const float* s_gate,
+                            const uint8_t* w_up, const float* s_up, const uint8_t* w_down, const float* s_down,
+                            float* y, float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws,
+                            size_t ws_bytes, void* stream, void* const* stage_events)
+{
+    return ffn_call(codes, act_scales, T, H, topk_ids, topk_w, top_k, expert_offsets, sorted_pairs, E, I, w_gate,
+                    s_gate, w_up, s_up, w_down, s_down, y, nullptr, 0, ws, ws_bytes, stream, stage_events, 1,
+                    routed_scaling, out_f32, out_bf16, "moe_grouped_ffn_combine");
 }
 
 size_t moe_combine_workspace_bytes(void) { return kStatusBytes; }

@@ -46,6 +46,7 @@
 // Every wait is bounded (2 s of global time); on expiry the CTA raises an
 // abort flag, records MOE_DEV_WAIT_TIMEOUT, drains and frees TMEM.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <cfloat>
@@ -139,6 +140,16 @@ struct GemmParams {
     int64_t y_nrows;
     int H;
     int* status;
+    // combine fused into the down epilogue (fuse = 1; items n-tile-major)
+    int ntmajor;
+    int fuse;
+    float rs;
+    float* out;                 // [T, H] FP32
+    uint16_t* out_bf16;         // nullable
+    int* cnt;                   // [T, n_tiles, 2] arrivals per token, n-tile and column half
+    const int32_t* topk_ids;    // [T, k]
+    const int32_t* nvalid;      // [T] valid slots per token
+    int k;
 };
 
 __device__ __forceinline__ int find_expert(const int* ipre, int E, int item)
@@ -159,9 +170,18 @@ struct Item {
 // Work items are ordered expert-major, then n-tile, then m-tile, so that the
 // m-tiles sharing a weight panel are processed at the same time by
 // neighbouring CTAs and share it in L2.
-__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item, int rev)
+__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item, int rev, int ntmajor)
 {
     Item it;
+    if (ntmajor) {  // n-tile-major: all m-tiles of every expert for one n-tile, then the next n-tile
+        const int mt_total = ipre[E];
+        it.nt = item / mt_total;
+        const int local = item - it.nt * mt_total;
+        const int o = find_expert(ipre, E, local);
+        it.e = rev ? E - 1 - o : o;
+        it.mt = local - ipre[o];
+        return it;
+    }
     const int o = find_expert(ipre, E, item);  // position of the expert in the walk order
     it.e = rev ? E - 1 - o : o;
     const int local = item - ipre[o];
@@ -184,7 +204,7 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
         const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
         const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
@@ -217,7 +237,7 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
         const int row0 = seg[w.e] + w.mt * BM;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             const int s = it % A_STAGES;
@@ -301,7 +321,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
     int it = 0;
     int nitem = 0;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++nitem) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev);
+        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
         const int r = seg[w.e] + w.mt * BM + trow;
         const bool valid = r < seg[w.e + 1];
         const int64_t ra = r < p.P ? r : p.P - 1;
@@ -328,6 +348,8 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                 yrow = p.y_rows ? __ldg(p.y_rows + pair) : pair;
             }
         }
+        int nval = 0;  // fused combine: valid slots of this row's token
+        if (MODE == 1 && p.fuse && pair >= 0 && pair < p.P) nval = __ldg(p.nvalid + pair / p.k);
 
         float acc0[64], acc1[64];
 #pragma unroll
@@ -443,6 +465,73 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                 }
                 if (half == 0) p.h_scales[static_cast<int64_t>(r) * p.GI + w.nt] = s;
             }
+        } else if (p.fuse) {
+            // Combine fused into the epilogue.  The row's two 64-column y
+            // segments are written, made visible, and counted on the
+            // (token, n-tile, column half) arrival counter; the thread whose
+            // arrival completes the token's valid slots marks that segment
+            // pair ready, and the whole warp then sums each ready token's
+            // slot rows in slot order (the combine's arithmetic: from zero,
+            // valid slots in order, times routed_scaling) with coalesced
+            // loads.  The order of arrival does not change any bit.
+            const bool mine = valid && pair >= 0 && pair < p.P;
+            if (valid && !mine) atomicOr(p.status, kDevBadPair);
+            const int c0 = w.nt * 256 + half * 64;
+            const int c1 = c0 + 128;
+            if (mine) {
+                float* dst = p.y + static_cast<int64_t>(pair) * p.H;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c = hh ? c1 : c0;
+                    if (c >= p.H) continue;
+                    const float* a = hh ? acc1 : acc0;
+                    float4* g = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+                    for (int q4 = 0; q4 < 16; ++q4)
+                        g[q4] = make_float4(wt * a[4 * q4], wt * a[4 * q4 + 1], wt * a[4 * q4 + 2], wt * a[4 * q4 + 3]);
+                }
+            }
+            __threadfence();
+            const int tok = mine ? pair / p.k : 0;
+            bool last = false;
+            if (mine) last = atomicAdd(p.cnt + (static_cast<int64_t>(tok) * p.n_tiles + w.nt) * 2 + half, 1) == nval - 1;
+            uint32_t ready = __ballot_sync(0xFFFFFFFFu, last);
+            if (ready) __threadfence();
+            while (ready) {
+                const int L = __ffs(ready) - 1;
+                ready &= ready - 1;
+                const int64_t t = __shfl_sync(0xFFFFFFFFu, tok, L);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c = (hh ? c1 : c0) + 2 * lane;  // this lane's two columns
+                    if ((hh ? c1 : c0) >= p.H) continue;
+                    float2 acc = make_float2(0.f, 0.f);
+                    for (int j0 = 0; j0 < p.k; j0 += 8) {
+                        float2 v[8];
+                        bool ok[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int j = j0 + u;
+                            const int e = (j < p.k) ? __ldg(p.topk_ids + t * p.k + j) : -1;
+                            ok[u] = e >= 0 && e < p.E;
+                            v[u] = ok[u] ? __ldcg(reinterpret_cast<const float2*>(p.y + (t * p.k + j) * p.H + c))
+                                         : make_float2(0.f, 0.f);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (!ok[u]) continue;
+                            acc.x += v[u].x;
+                            acc.y += v[u].y;
+                        }
+                    }
+                    const float2 o = make_float2(p.rs * acc.x, p.rs * acc.y);
+                    *reinterpret_cast<float2*>(p.out + t * p.H + c) = o;
+                    if (p.out_bf16) {
+                        const __nv_bfloat162 bb = __floats2bfloat162_rn(o.x, o.y);
+                        *reinterpret_cast<__nv_bfloat162*>(p.out_bf16 + t * p.H + c) = bb;
+                    }
+                }
+            }
         } else {
             if (valid) {
                 if (pair < 0 || pair >= p.P || yrow >= p.y_nrows) {
@@ -535,7 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int c = seg[e + 1] - seg[e];
             if (c < 0 || seg[e + 1] > p.P) okv = 0;
             const int mts = c > 0 ? (c + BM - 1) / BM : 0;
-            acc += mts * p.n_tiles;
+            acc += p.ntmajor ? mts : mts * p.n_tiles;
             ipre[o + 1] = acc;
         }
         if (!okv) {
@@ -547,7 +636,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total_items = *bad ? 0 : ipre[E];
+    const int total_items = *bad ? 0 : (p.ntmajor ? ipre[E] * p.n_tiles : ipre[E]);
 
     if (warp < 4) {
         setmaxnreg_dec<REGS_CTRL>();
@@ -612,6 +701,32 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
     }
 }
 
+// Fused combine, before the GEMMs: per token (one warp each), zero the
+// arrival counters, count the valid slots, and write the zero row of a token
+// with none (no arrival will come for it).
+__global__ void __launch_bounds__(256) fuse_prep_kernel(const int32_t* __restrict__ ids, int64_t T, int k, int E,
+                                                        int n_tiles, int H, int* __restrict__ cnt,
+                                                        int32_t* __restrict__ nvalid, float* __restrict__ out,
+                                                        uint16_t* __restrict__ out_bf16)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    for (int i = lane; i < n_tiles * 2; i += 32) cnt[t * n_tiles * 2 + i] = 0;
+    int n = 0;
+    for (int j = 0; j < k; ++j) {
+        const int e = __ldg(ids + t * k + j);
+        n += (e >= 0 && e < E) ? 1 : 0;
+    }
+    if (lane == 0) nvalid[t] = n;
+    if (n == 0) {
+        for (int c = lane; c < H; c += 32) {
+            out[t * H + c] = 0.f;
+            if (out_bf16) out_bf16[t * H + c] = 0;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
@@ -673,7 +788,7 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 }  // namespace
 
 size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
-                            size_t* off_sh)
+                            size_t* off_sh, size_t* off_cnt, size_t* off_nv)
 {
     const int64_t P = T * k > 0 ? T * k : 1;
     const int GI = (I + 127) / 128;
@@ -687,6 +802,13 @@ size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_
     o = align_up(o + static_cast<size_t>(P) * Ip, 256);
     *off_sh = o;
     o = align_up(o + static_cast<size_t>(P) * GI * 4, 256);
+    // fused combine: arrival counters [T, ceil(H/256), 2], valid slots [T]
+    const size_t t = static_cast<size_t>(T > 0 ? T : 1);
+    size_t dummy;
+    (off_cnt ? *off_cnt : dummy) = o;
+    o = align_up(o + t * ((H + 255) / 256) * 2 * 4, 256);
+    (off_nv ? *off_nv : dummy) = o;
+    o = align_up(o + t * 4, 256);
     return o;
 }
 
@@ -775,6 +897,23 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     d.b_s1 = a.s_down;
     d.b_nblocks = GH;
     d.rev = 0;
+    if (a.fuse) {
+        // prep (counters, valid slots, empty rows), then the down items
+        // n-tile-major so that a token's slot rows meet in L2
+        const int nt_down = (H + 255) / 256;
+        fuse_prep_kernel<<<static_cast<int>(ceil_div64(a.T * 32, 256)), 256, 0, s>>>(
+            a.topk_ids, a.T, a.k, E, nt_down, H, a.cnt, a.nvalid, a.out, a.out_bf16);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        d.ntmajor = 1;
+        d.fuse = 1;
+        d.rs = a.rs;
+        d.out = a.out;
+        d.out_bf16 = a.out_bf16;
+        d.cnt = a.cnt;
+        d.topk_ids = a.topk_ids;
+        d.nvalid = a.nvalid;
+        d.k = a.k;
+    }
     if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
     if ((err = run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;
     return stage_mark(a, 3, s);

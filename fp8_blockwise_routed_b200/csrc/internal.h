@@ -120,9 +120,16 @@ struct FfnArgs {
     uint8_t* h_codes;    // [P, Ip]
     float* h_scales;     // [P, ceil(I/128)]
     void* const* stage_events;  // nullable: 4 cudaEvent_t for profiling
+    // combine fused into the down GEMM (fuse = 1): out = rs * slot sum
+    int fuse;
+    float rs;
+    float* out;            // [T, H]
+    uint16_t* out_bf16;    // nullable
+    int* cnt;              // workspace: arrival counters
+    int32_t* nvalid;       // workspace: valid slots per token
 };
 size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
-                            size_t* off_sh);
+                            size_t* off_sh, size_t* off_cnt = nullptr, size_t* off_nv = nullptr);
 // Returns cudaSuccess, or an error (including cudaErrorNotSupported when the
 // tensor-map encoder cannot be obtained).
 cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s);

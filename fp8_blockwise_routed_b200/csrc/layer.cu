@@ -72,7 +72,7 @@ struct LayerArgs {
 
 // The three calls; stage events (nullable, 6): start, then the four marks of
 // moe_grouped_ffn (gather, gate/up, down, down end), then the end.
-int run_layer(const LayerArgs& a, cudaStream_t s, void* const* ev)
+int run_layer(const LayerArgs& a, cudaStream_t s, void* const* ev, int flags = 0)
 {
     LayerLayout L;
     if (!layer_layout(a.T, a.H, a.I, a.E, a.top_k, &L)) return MOE_ERR_INVALID_ARG;
@@ -90,11 +90,22 @@ int run_layer(const LayerArgs& a, cudaStream_t s, void* const* ev)
     int r = moe_route_quant(a.logits, a.x, a.T, a.H, a.E, a.top_k, ids, tw, offsets, sorted, codes, scales,
                             w + L.route, L.ffn - L.route, s);
     if (r) return r;
-    r = moe_grouped_ffn(codes, scales, a.T, a.H, ids, tw, a.top_k, offsets, sorted, a.E, a.I, a.w_gate, a.s_gate,
-                        a.w_up, a.s_up, a.w_down, a.s_down, y, w + L.ffn, L.comb - L.ffn, s, ev ? ev + 1 : nullptr);
-    if (r) return r;
-    r = moe_combine(y, ids, a.T, a.H, a.top_k, a.E, a.rs, a.out_f32, a.out_bf16, w + L.comb, L.codes - L.comb, s);
-    if (r) return r;
+    if (flags & MOE_LAYER_FUSED_COMBINE) {
+        r = moe_grouped_ffn_combine(codes, scales, a.T, a.H, ids, tw, a.top_k, offsets, sorted, a.E, a.I, a.w_gate,
+                                    a.s_gate, a.w_up, a.s_up, a.w_down, a.s_down, y, a.rs, a.out_f32, a.out_bf16,
+                                    w + L.ffn, L.comb - L.ffn, s, ev ? ev + 1 : nullptr);
+        if (r) return r;
+        // no separate combine runs: its status word stays clear
+        if (cudaMemsetAsync(w + L.comb, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        r = moe_grouped_ffn(codes, scales, a.T, a.H, ids, tw, a.top_k, offsets, sorted, a.E, a.I, a.w_gate,
+                            a.s_gate, a.w_up, a.s_up, a.w_down, a.s_down, y, w + L.ffn, L.comb - L.ffn, s,
+                            ev ? ev + 1 : nullptr);
+        if (r) return r;
+        r = moe_combine(y, ids, a.T, a.H, a.top_k, a.E, a.rs, a.out_f32, a.out_bf16, w + L.comb, L.codes - L.comb,
+                        s);
+        if (r) return r;
+    }
     if (ev && fp8moe::record_event(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -128,6 +139,17 @@ int moe_layer_plan_create(moe_layer_plan** plan, const float* logits, const uint
                           const float* s_up, const uint8_t* w_down, const float* s_down, float routed_scaling,
                           float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes, void* const* stage_events)
 {
+    return moe_layer_plan_create_ex(plan, logits, x, T, H, E, top_k, I, w_gate, s_gate, w_up, s_up, w_down, s_down,
+                                    routed_scaling, out_f32, out_bf16, ws, ws_bytes, stage_events, 0);
+}
+
+int moe_layer_plan_create_ex(moe_layer_plan** plan, const float* logits, const uint16_t* x, int64_t T, int H, int E,
+                             int top_k, int I, const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
+                             const float* s_up, const uint8_t* w_down, const float* s_down, float routed_scaling,
+                             float* out_f32, uint16_t* out_bf16, void* ws, size_t ws_bytes, void* const* stage_events,
+                             int flags)
+{
+    if (flags & ~MOE_LAYER_FUSED_COMBINE) return MOE_ERR_INVALID_ARG;
     if (!plan) return MOE_ERR_INVALID_ARG;
     *plan = nullptr;
     const LayerArgs a{logits, x,    T,    H,     E,     top_k,          I,        w_gate, s_gate,
@@ -139,7 +161,7 @@ int moe_layer_plan_create(moe_layer_plan** plan, const float* logits, const uint
         cudaStreamDestroy(cs);
         return MOE_ERR_CUDA;
     }
-    const int r = run_layer(a, cs, stage_events);
+    const int r = run_layer(a, cs, stage_events, flags);
     cudaGraph_t graph = nullptr;
     const cudaError_t end = cudaStreamEndCapture(cs, &graph);
     cudaStreamDestroy(cs);

@@ -281,6 +281,29 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_grouped_ffn_combine -- moe_grouped_ffn with moe_combine fused into the
+ * down GEMM's epilogue (the plan's first "next" step).  Arguments as
+ * moe_grouped_ffn (y is still written: it carries the slot rows between the
+ * GEMM's tiles) plus routed_scaling, out_f32 [T, H] and out_bf16 (nullable) as
+ * moe_combine.  The down items run n-tile-major, so a token's k slot rows of
+ * one 256-column block are produced close together.  Each slot row segment
+ * counts an arrival per (token, n-tile, column half); the arrival that
+ * completes a token's valid slots makes its warp sum the token's slot rows in
+ * slot order.  The arithmetic is moe_combine's (from zero, valid slots in
+ * order, times routed_scaling), so the result equals moe_grouped_ffn followed
+ * by moe_combine bit for bit, whatever the order of arrival.  Rows of tokens
+ * without a valid slot are written as zeros.  Workspace:
+ * moe_ffn_workspace_bytes (it includes the arrival counters).
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_grouped_ffn_combine(const uint8_t* codes, const float* act_scales, int64_t T, int H,
+                                    const int32_t* topk_ids, const float* topk_w, int top_k,
+                                    const int32_t* expert_offsets, const int32_t* sorted_pairs, int E, int I,
+                                    const uint8_t* w_gate, const float* s_gate, const uint8_t* w_up,
+                                    const float* s_up, const uint8_t* w_down, const float* s_down, float* y,
+                                    float routed_scaling, float* out_f32, uint16_t* out_bf16, void* ws,
+                                    size_t ws_bytes, void* stream, void* const* stage_events);
+
+/* ---------------------------------------------------------------------------
  * Shared-expert slot.  The pages plan a shared expert as one more slot after
  * the routed ones ("GLM-5.3-Flash EXL3 on CUDA ...": all nine slots planned
  * with E+1 expert ids, the shared id skipped before any routed payload is
@@ -404,6 +427,16 @@ MOE_API int moe_layer_plan_create(moe_layer_plan** plan, const float* logits, co
                                   const uint8_t* w_up, const float* s_up, const uint8_t* w_down,
                                   const float* s_down, float routed_scaling, float* out_f32, uint16_t* out_bf16,
                                   void* ws, size_t ws_bytes, void* const* stage_events);
+/* moe_layer_plan_create with options: flags = MOE_LAYER_FUSED_COMBINE uses
+ * moe_grouped_ffn_combine in place of moe_grouped_ffn + moe_combine (the
+ * stage events then mark the start, the gather, gate/up and down launches,
+ * the end of the fused down launch, and the end). */
+#define MOE_LAYER_FUSED_COMBINE 1
+MOE_API int moe_layer_plan_create_ex(moe_layer_plan** plan, const float* logits, const uint16_t* x, int64_t T,
+                                     int H, int E, int top_k, int I, const uint8_t* w_gate, const float* s_gate,
+                                     const uint8_t* w_up, const float* s_up, const uint8_t* w_down,
+                                     const float* s_down, float routed_scaling, float* out_f32, uint16_t* out_bf16,
+                                     void* ws, size_t ws_bytes, void* const* stage_events, int flags);
 MOE_API int moe_layer_plan_launch(moe_layer_plan* plan, void* stream);
 MOE_API void moe_layer_plan_destroy(moe_layer_plan* plan);
 MOE_API int moe_layer_get_device_status(const void* ws, int64_t T, int H, int I, int E, int top_k,
