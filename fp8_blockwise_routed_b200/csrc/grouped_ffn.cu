@@ -140,9 +140,7 @@ struct GemmParams {
     int64_t y_nrows;
     int H;
     int* status;
-    // combine fused into the down epilogue (fuse = 1; items n-tile-major)
-    int ntmajor;
-    int fuse;
+    // combine fused into the down epilogue (MODE 2; items n-tile-major)
     float rs;
     float* out;                 // [T, H] FP32
     uint16_t* out_bf16;         // nullable
@@ -170,10 +168,11 @@ struct Item {
 // Work items are ordered expert-major, then n-tile, then m-tile, so that the
 // m-tiles sharing a weight panel are processed at the same time by
 // neighbouring CTAs and share it in L2.
-__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item, int rev, int ntmajor)
+template <bool NTMAJOR>
+__device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int E, int item, int rev)
 {
     Item it;
-    if (ntmajor) {  // n-tile-major: all m-tiles of every expert for one n-tile, then the next n-tile
+    if (NTMAJOR) {  // n-tile-major: all m-tiles of every expert for one n-tile, then the next n-tile
         const int mt_total = ipre[E];
         it.nt = item / mt_total;
         const int local = item - it.nt * mt_total;
@@ -204,7 +203,7 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
+        const Item w = decode_item<MODE == 2>(seg, ipre, p.E, item, p.rev);
         const int n0 = (MODE == 0) ? w.nt * 128 : w.nt * 256;
         const int n1 = (MODE == 0) ? w.nt * 128 : w.nt * 256 + 128;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
@@ -230,6 +229,7 @@ __device__ __forceinline__ void producer_b(const CUtensorMap* tmB0, const CUtens
 
 // Activation producer (one lane): the 128-row A tile of every K block into
 // an A_STAGES-deep ring.
+template <int MODE>
 __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmParams& p, const int* seg,
                                            const int* ipre, int total_items, uint32_t sbase, uint32_t bars,
                                            volatile int* abort)
@@ -237,7 +237,7 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
     int it = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
+        const Item w = decode_item<MODE == 2>(seg, ipre, p.E, item, p.rev);
         const int row0 = seg[w.e] + w.mt * BM;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             const int s = it % A_STAGES;
@@ -321,7 +321,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
     int it = 0;
     int nitem = 0;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++nitem) {
-        const Item w = decode_item(seg, ipre, p.E, item, p.rev, p.ntmajor);
+        const Item w = decode_item<MODE == 2>(seg, ipre, p.E, item, p.rev);
         const int r = seg[w.e] + w.mt * BM + trow;
         const bool valid = r < seg[w.e + 1];
         const int64_t ra = r < p.P ? r : p.P - 1;
@@ -341,7 +341,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
         int pair = -1;
         int64_t yrow = -1;
         float wt = 0.f;
-        if (MODE == 1 && valid) {
+        if (MODE != 0 && valid) {
             pair = __ldg(p.sorted_pairs + r);
             if (pair >= 0 && pair < p.P) {
                 wt = __ldg(p.topk_w + pair);
@@ -349,7 +349,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             }
         }
         int nval = 0;  // fused combine: valid slots of this row's token
-        if (MODE == 1 && p.fuse && pair >= 0 && pair < p.P) nval = __ldg(p.nvalid + pair / p.k);
+        if (MODE == 2 && pair >= 0 && pair < p.P) nval = __ldg(p.nvalid + pair / p.k);
 
         float acc0[64], acc1[64];
 #pragma unroll
@@ -465,7 +465,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                 }
                 if (half == 0) p.h_scales[static_cast<int64_t>(r) * p.GI + w.nt] = s;
             }
-        } else if (p.fuse) {
+        } else if (MODE == 2) {
             // Combine fused into the epilogue.  The row's two 64-column y
             // segments are written, made visible, and counted on the
             // (token, n-tile, column half) arrival counter; the thread whose
@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int c = seg[e + 1] - seg[e];
             if (c < 0 || seg[e + 1] > p.P) okv = 0;
             const int mts = c > 0 ? (c + BM - 1) / BM : 0;
-            acc += p.ntmajor ? mts : mts * p.n_tiles;
+            acc += (MODE == 2) ? mts : mts * p.n_tiles;
             ipre[o + 1] = acc;
         }
         if (!okv) {
@@ -636,21 +636,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total_items = *bad ? 0 : (p.ntmajor ? ipre[E] * p.n_tiles : ipre[E]);
+    const int total_items = *bad ? 0 : ((MODE == 2) ? ipre[E] * p.n_tiles : ipre[E]);
 
     if (warp < 4) {
         setmaxnreg_dec<REGS_CTRL>();
         if ((threadIdx.x & 31) == 0) {
             if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
             else if (warp == 1 || warp == 2) mma_role<MODE>(p, total_items, sbase, bars, tmem, abort, warp - 1);
-            else if (warp == 3) producer_a(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
+            else if (warp == 3) producer_a<MODE>(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {
         setmaxnreg_inc<REGS_EPI>();
         epilogue_role<MODE>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
         // the y bulk copies must be done with shared memory (and complete)
         // before the CTA exits
-        if (MODE == 1) bulk_wait_all();
+        if (MODE != 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -804,10 +804,9 @@ size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_
     o = align_up(o + static_cast<size_t>(P) * GI * 4, 256);
     // fused combine: arrival counters [T, ceil(H/256), 2], valid slots [T]
     const size_t t = static_cast<size_t>(T > 0 ? T : 1);
-    size_t dummy;
-    (off_cnt ? *off_cnt : dummy) = o;
+    if (off_cnt) *off_cnt = o;
     o = align_up(o + t * ((H + 255) / 256) * 2 * 4, 256);
-    (off_nv ? *off_nv : dummy) = o;
+    if (off_nv) *off_nv = o;
     o = align_up(o + t * 4, 256);
     return o;
 }
@@ -904,8 +903,6 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
         fuse_prep_kernel<<<static_cast<int>(ceil_div64(a.T * 32, 256)), 256, 0, s>>>(
             a.topk_ids, a.T, a.k, E, nt_down, H, a.cnt, a.nvalid, a.out, a.out_bf16);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
-        d.ntmajor = 1;
-        d.fuse = 1;
         d.rs = a.rs;
         d.out = a.out;
         d.out_bf16 = a.out_bf16;
@@ -915,7 +912,9 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
         d.k = a.k;
     }
     if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
-    if ((err = run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;
+    if ((err = a.fuse ? run_gemm<2>(tmA2, tmD, tmD, d, grid, s) : run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) !=
+        cudaSuccess)
+        return err;
     return stage_mark(a, 3, s);
 }
 
