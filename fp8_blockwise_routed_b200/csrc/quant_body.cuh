@@ -2,8 +2,10 @@
 // quant_act_kernel and the fused route+quantise launch.
 //
 // Rule per 1x128 group: amax = max|x|; s = amax/448 (IEEE divide); s == 0 ->
-// 1; code = E4M3_rn_satfinite(x/s) (IEEE divide); a group holding NaN/Inf
-// gets s = NaN and codes 0x7F.  No flush-to-zero (built without fast-math).
+// 1; code = E4M3_rn_satfinite(x/s) (the IEEE quotient, formed below by a
+// corrected reciprocal product that yields the same codes); a group holding
+// NaN/Inf gets s = NaN and codes 0x7F.  No flush-to-zero (built without
+// fast-math).
 //
 // A half-warp owns one group: each lane loads one 16-byte vector (8 BF16),
 // the 16 lanes reduce amax with shuffles, each lane stores 8 code bytes, lane
@@ -26,6 +28,24 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p)
 }
 
 constexpr int kUnroll = 4;  // groups per half-warp per trip, loads issued together
+
+// x / s without the divide: with y = RN(1/s) and q = RN(x*y), the remainder
+// r = s*q - x is exact in one FMA and RN(q - r*y) is the correctly rounded
+// quotient (Markstein's correction step, P. Markstein, IBM J. Res. Dev.
+// 34(1), 1990), as long as r does not underflow.  For BF16 x and
+// s = RN(amax/448) with |x| <= amax, an exhaustive comparison with the IEEE
+// divide over every such pair with s >= 2^-100 finds equal E4M3 codes
+// everywhere: the two floats differ only where both are below 2^-11 in
+// magnitude, i.e. both encode to zero.  The sign is copied from x so that
+// zero quotients keep it (-0/s = -0).  Smaller scales keep the divide.
+constexpr float kExactQuotientMinScale = 0x1p-100f;
+
+__device__ __forceinline__ float quotient(float x, float s, float y)
+{
+    const float q = __fmul_rn(x, y);
+    const float r = __fmaf_rn(s, q, -x);
+    return copysignf(__fmaf_rn(-r, y, q), x);
+}
 
 // Quantises groups [0, n_groups) with the warps of `nblocks` blocks of
 // blockDim.x threads, this thread belonging to block `block`.  Per trip a
@@ -75,7 +95,16 @@ __device__ __forceinline__ void groups(const uint4* __restrict__ x, int64_t n_gr
             if (bad) {
                 s = __int_as_float(0x7FC00000);
                 out = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
-            } else {
+            } else if (s >= kExactQuotientMinScale) {
+                const float y = __frcp_rn(s);
+                float d[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) d[i] = quotient(v[i], s, y);
+                uint32_t p[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) p[i] = sm100::e4m3x2(d[2 * i], d[2 * i + 1]);
+                out = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+            } else {  // groups whose amax is below 448 * 2^-100
                 uint32_t p[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)

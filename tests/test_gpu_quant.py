@@ -83,3 +83,42 @@ def test_quant_act_rejects_bad_width():
         fm.moe_quant_act(x, torch.empty((4, 200), dtype=torch.uint8, device="cuda"),
                          torch.empty((4, 2), dtype=torch.float32, device="cuda"))
     assert e.value.code == 1
+
+
+def test_quant_act_every_amax_mantissa_across_binades():
+    """Groups whose maximum is each of the 128 BF16 mantissas at amax
+    exponents from the subnormals through the largest binade, including
+    both sides of amax = 448 * 2^-100 (where the kernel switches between its
+    divide-free quotient and the divide).  The other 127 values of a group are
+    random BF16 patterns of magnitude <= amax spread over 40 binades below it,
+    with signed zeros.  Codes and scales bit-exact against the oracle."""
+    rng = np.random.default_rng(11)
+    exps = [0, 1, 2, 30, 33, 34, 35, 36, 37, 38, 60, 100, 120, 126, 127, 128, 135, 200, 240, 253, 254]
+    groups = []
+    for e in exps:
+        for m in range(128):
+            if e == 0 and m == 0:
+                continue
+            amax = (e << 7) | m
+            lo = max(0, e - 40)
+            ex = rng.integers(lo, e + 1, size=127)
+            mant = rng.integers(0, 128, size=127)
+            top = ex == e
+            mant[top] = rng.integers(0, m + 1, size=int(top.sum()))
+            mag = (ex << 7) | mant
+            mag[rng.random(127) < 0.03] = 0
+            g = np.concatenate([[amax], mag]).astype(np.uint16)
+            g |= (rng.random(128) < 0.5).astype(np.uint16) << 15
+            rng.shuffle(g)
+            groups.append(g)
+    n = len(groups)
+    per_row = 8
+    n_rows = (n + per_row - 1) // per_row
+    bits = np.zeros((n_rows * per_row, 128), np.uint16)
+    bits[:n] = np.stack(groups)
+    bits = bits.reshape(n_rows, per_row * 128)
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, scales = _quant(x)
+    rc, rs = oracle.quant_act(x.cpu())
+    assert np.array_equal(codes, rc)
+    assert np.array_equal(scales.view(np.uint32), rs.view(np.uint32))
