@@ -1,11 +1,11 @@
 // quant_body.cuh -- the activation quantiser's per-group body, shared by
 // quant_act_kernel and the fused route+quantise launch.
 //
-// Rule per 1x128 group: amax = max|x|; s = amax/448 (IEEE divide); s == 0 ->
-// 1; code = E4M3_rn_satfinite(x/s) (the IEEE quotient, formed below by a
-// corrected reciprocal product that yields the same codes); a group holding
-// NaN/Inf gets s = NaN and codes 0x7F.  No flush-to-zero (built without
-// fast-math).
+// Rule per 1x128 group: amax = max|x|; s = amax/448 (the IEEE quotient);
+// s == 0 -> 1; code = E4M3_rn_satfinite(x/s) (the IEEE quotient); a group
+// holding NaN/Inf gets s = NaN and codes 0x7F.  Both quotients are formed
+// below without a divide, by corrected reciprocal products that give the
+// same scales and codes.  No flush-to-zero (built without fast-math).
 //
 // A half-warp owns one group: each lane loads one 16-byte vector (8 BF16),
 // the 16 lanes reduce amax with shuffles, each lane stores 8 code bytes, lane
@@ -47,6 +47,19 @@ __device__ __forceinline__ float quotient(float x, float s, float y)
     return copysignf(__fmaf_rn(-r, y, q), x);
 }
 
+// s = RN(amax / 448) by the same correction with y = RN(1/448): for every
+// finite non-negative BF16 amax (the group maximum is one of the group's
+// BF16 values) it equals the IEEE quotient, subnormal results included
+// (exhaustive host comparison over all 32,640 values).
+constexpr float kInv448 = 0x1.24924ap-9f;
+
+__device__ __forceinline__ float group_scale(float amax)
+{
+    const float q = __fmul_rn(amax, kInv448);
+    const float r = __fmaf_rn(448.0f, q, -amax);
+    return __fmaf_rn(-r, kInv448, q);
+}
+
 // Quantises groups [0, n_groups) with the warps of `nblocks` blocks of
 // blockDim.x threads, this thread belonging to block `block`.  Per trip a
 // warp covers 2*kUnroll consecutive groups; its loads are issued before any
@@ -77,19 +90,16 @@ __device__ __forceinline__ void groups(const uint4* __restrict__ x, int64_t n_gr
                 v[2 * i] = __uint_as_float(w[i] << 16);
                 v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
             }
+            // NaN-propagating max: a NaN or Inf anywhere in the group leaves
+            // amax non-finite, so one test after the reduction finds it
             float amax = 0.0f;
-            int bad = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (isfinite(v[i])) amax = fmaxf(amax, fabsf(v[i]));
-                else bad = 1;
-            }
+            for (int i = 0; i < 8; ++i) amax = sm100::fmax_nan(amax, fabsf(v[i]));
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) {
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-                bad |= __shfl_xor_sync(0xFFFFFFFFu, bad, off);
-            }
-            float s = __fdiv_rn(amax, 448.0f);
+            for (int off = 8; off > 0; off >>= 1)
+                amax = sm100::fmax_nan(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+            const bool bad = !isfinite(amax);
+            float s = group_scale(amax);
             if (s == 0.0f) s = 1.0f;
             uint2 out;
             if (bad) {

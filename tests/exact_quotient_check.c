@@ -9,8 +9,11 @@
  * this program compares d with the IEEE quotient RN(x/s) and counts the
  * pairs whose E4M3 codes could differ: d != RN(x/s) unless both lie below
  * 2^-11 in magnitude with the same sign (E4M3 encodes every magnitude below
- * 2^-10 to a signed zero).  It prints "pairs=<n> code_mismatch=<m>
- * float_mismatch=<f>" and exits 0. */
+ * 2^-10 to a signed zero).  The group scale itself is formed the same way,
+ * with y = RN(1/448); for every finite non-negative BF16 amax the program
+ * compares it with RN(amax/448) bit for bit.  It prints "pairs=<n>
+ * code_mismatch=<m> float_mismatch=<f> scales=<s> scale_mismatch=<z>" and
+ * exits 0. */
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -57,6 +60,19 @@ int main(void)
             }
         }
     }
-    printf("pairs=%lld code_mismatch=%lld float_mismatch=%lld\n", pairs, code_bad, float_bad);
+    long long scales = 0, scale_bad = 0;
+    volatile float inv448v = 1.0f / 448.0f;
+    const float inv448 = inv448v;
+    for (int ai = 0; ai < 0x7F80; ++ai) {
+        const float amax = bf16((uint32_t)ai);
+        volatile float div = amax / 448.0f;
+        volatile float q = amax * inv448;
+        volatile float r = fmaf(448.0f, q, -amax);
+        volatile float d = fmaf(-r, inv448, q);
+        ++scales;
+        if (bits(div) != bits(d)) ++scale_bad;
+    }
+    printf("pairs=%lld code_mismatch=%lld float_mismatch=%lld scales=%lld scale_mismatch=%lld\n", pairs, code_bad,
+           float_bad, scales, scale_bad);
     return 0;
 }
