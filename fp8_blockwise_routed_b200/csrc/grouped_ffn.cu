@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cfloat>
 #include <cstring>
 #include <mutex>
@@ -772,14 +773,15 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
                      int grid, cudaStream_t s)
 {
     const int smem = smem_bytes_for(MAX_E);
-    static bool attr_done[64] = {};
+    // per device, once; host threads may launch concurrently
+    static std::atomic<bool> attr_done[64];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
+        err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
-        attr_done[dev] = true;
+        if (dev < 64) attr_done[dev].store(true, std::memory_order_release);
     }
     grouped_gemm_kernel<MODE><<<grid, THREADS, smem_bytes_for(p.E), s>>>(a, b0, b1, p);
     return cudaGetLastError();
