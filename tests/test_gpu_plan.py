@@ -98,3 +98,31 @@ def test_plan_rejects_bad_arguments_without_capturing():
     torch.cuda.synchronize()
     assert plan.device_status() == 0
     plan.close()
+
+
+@pytest.mark.parametrize("T,H,E,k,I", [
+    (37, 640, 5, 1, 192),     # odd group count per token (5), T not a multiple of 8 tokens per block, k = 1
+    (203, 1024, 12, 3, 320),  # k = 3, several 128-row tiles with ragged tails
+    (1, 256, 4, 4, 128),      # one token, every expert taken
+])
+def test_layer_edge_shapes_equal_three_calls(T, H, E, k, I):
+    """The layer's route writes the activation codes straight into the
+    expert-ordered A rows (no gather): bit-identical to the separate calls
+    on edge shapes, with fully masked tokens (every slot empty) and a NaN
+    token among them."""
+    wl = mi.Workload("edge", T, H, E, k, I, 1.5, "normal", "normal")
+    d = mi.make_inputs(wl, 3, "cuda")
+    if T > 2:
+        d["logits"][1] = float("-inf")       # a token with no selectable expert
+        d["logits"][T - 1, :] = float("-inf")
+        d["x"][T // 2, 7] = float("nan")      # NaN stays in its token's row
+    ref = _three_calls(wl, d)
+    out = torch.full_like(ref, 7.0)
+    ws = torch.empty((fm.moe_layer_workspace_bytes(T, H, I, E, k),), dtype=torch.uint8, device="cuda")
+    fm.moe_layer(d["logits"], d["x"], k, *_w(d), wl.routed_scaling, out, None, ws)
+    torch.cuda.synchronize()
+    assert fm.moe_layer_get_device_status(ws, T, H, I, E, k) == 0
+    assert torch.equal(out.view(torch.int32), ref.view(torch.int32))
+    if T > 2:
+        assert torch.all(out[1] == 0) and torch.all(out[T - 1] == 0)
+        assert torch.isnan(out[T // 2]).all()
