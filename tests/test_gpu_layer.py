@@ -23,6 +23,9 @@ SMALL = {
     "h640": mi.Workload("h640", 333, 640, 12, 4, 320, 0.5, "normal", "uniform"),
     # one expert, top-1: a dense FFN
     "dense": mi.Workload("dense", 150, 256, 1, 1, 256, 1.0, "normal", "normal"),
+    # the largest hidden and intermediate widths the ABI accepts (H 16384,
+    # I 8192: 128 K blocks for gate/up, 64 for down, 64 N tiles each)
+    "maxdims": mi.Workload("maxdims", 16, 16384, 3, 2, 8192, 1.0, "normal", "normal"),
 }
 
 
