@@ -26,6 +26,9 @@ SMALL = {
     # the largest hidden and intermediate widths the ABI accepts (H 16384,
     # I 8192: 128 K blocks for gate/up, 64 for down, 64 N tiles each)
     "maxdims": mi.Workload("maxdims", 16, 16384, 3, 2, 8192, 1.0, "normal", "normal"),
+    # the most experts and slots the ABI accepts (E 1024, top-32): ~2 rows
+    # per expert, one partly filled tile each, 32 slot rows per token
+    "maxexperts": mi.Workload("maxexperts", 64, 256, 1024, 32, 128, 1.0, "normal", "normal"),
 }
 
 
