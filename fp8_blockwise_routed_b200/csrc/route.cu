@@ -27,6 +27,8 @@
 //      rank_in_block(p); positions past offsets[E] get -1.
 // Every integer output is a pure function of the ids, so it is the same for
 // any launch shape and from run to run.
+#include <cuda.h>
+
 #include <cfloat>
 #include <climits>
 #include <cstdio>
@@ -346,24 +348,64 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = (size_t(1) << 20) + 4096;
 __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
 
-// Device address of g_route_scratch, looked up once per device with that
-// device current (in host code the symbol is only a host-side stand-in and
-// must not be passed to a kernel).
+// Identity of the calling thread's current CUDA context (the driver's
+// cuCtxGetCurrent and cuCtxGetId, reached through the runtime's entry-point
+// query so that libcuda need not be linked).  A device reset, or the release
+// and re-creation of the primary context, gives a new id, and with it new
+// module addresses.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id)
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_route_scratch in the current context.  In host code the
+// symbol is only a host-side stand-in and must not be passed to a kernel.
+// The address is looked up (cudaGetSymbolAddress) the first time a context
+// calls, with its device current, and cached per device together with the
+// context's id; a call from a different context (after a device reset, for
+// instance) looks it up again, so a stale address is never used.
 void* scratch_address(int dev, cudaError_t* err)
 {
     static void* addr[64] = {};
+    static unsigned long long ctx_of[64] = {};
     static std::mutex mu;
-    std::lock_guard<std::mutex> lk(mu);
     *err = cudaSuccess;
     if (dev < 0 || dev >= 64) {
         *err = cudaErrorInvalidDevice;
         return nullptr;
     }
-    if (!addr[dev]) {
+    std::lock_guard<std::mutex> lk(mu);
+    unsigned long long ctx = 0;
+    const bool known = current_context_id(&ctx);  // false before the runtime made a context current
+    if (!known || !addr[dev] || ctx_of[dev] != ctx) {
         void* p = nullptr;
-        *err = cudaGetSymbolAddress(&p, g_route_scratch);
+        *err = cudaGetSymbolAddress(&p, g_route_scratch);  // creates the context if there was none
         if (*err != cudaSuccess) return nullptr;
+        if (!current_context_id(&ctx)) {
+            *err = cudaErrorDeviceUninitialized;
+            return nullptr;
+        }
         addr[dev] = p;
+        ctx_of[dev] = ctx;
     }
     return addr[dev];
 }
@@ -381,6 +423,8 @@ extern "C" int moe_route_noalloc(const float* logits, int64_t T, int E, int top_
     g_noalloc_error[0] = 0;
     if (T < 0 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 0 || top_k > E || top_k > MOE_MAX_TOP_K)
         return MOE_ERR_INVALID_ARG;
+    // moe_route's cap on T (int32 pair indices), before any size arithmetic
+    if (T > (int64_t(1) << 31) / (top_k > 0 ? top_k : 1) - 1) return MOE_ERR_UNSUPPORTED;
     if (!expert_offsets) return MOE_ERR_INVALID_ARG;
     if (T > 0 && top_k > 0 && (!logits || !topk_ids || !topk_w || !sorted_pairs)) return MOE_ERR_INVALID_ARG;
     auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
