@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
         L.moe_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         L.moe_debug_encode.restype = i32
         L.moe_debug_encode.argtypes = [P, i64, P, P]
+        L.moe_debug_grouped_down.restype = i32
+        L.moe_debug_grouped_down.argtypes = [P, P, i64, i32, i32, P, P, P, i32, i32, P, P, P, P, sz, P]
         L.moe_ffn_intermediate.restype = i32
         L.moe_ffn_intermediate.argtypes = [P, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p),
                                            ctypes.POINTER(ctypes.c_void_p)]
@@ -235,6 +237,18 @@ def moe_ffn_intermediate(ws, T: int, H: int, I: int, top_k: int):
     codes = ws[oc: oc + P * GI * 128].view(P, GI * 128)
     scales = ws[osc: osc + P * GI * 4].view(torch.float32).view(P, GI)
     return codes, scales
+
+
+def moe_debug_grouped_down(h_codes, h_scales, topk_w, expert_offsets, sorted_pairs, w_down, s_down, y, ws,
+                           stream=None):
+    """Test hook: the down GEMM alone on a caller-supplied intermediate
+    (h_codes [T*top_k, Ip] uint8, h_scales [T*top_k, ceil(I/128)] float32,
+    rows in expert order), writing y [T, top_k, H] for the valid pairs."""
+    T, k = topk_w.shape
+    E, H, I = w_down.shape
+    _check(lib().moe_debug_grouped_down(_p(h_codes), _p(h_scales), T, H, k, _p(topk_w), _p(expert_offsets),
+                                        _p(sorted_pairs), E, I, _p(w_down), _p(s_down), _p(y), _p(ws),
+                                        ws.numel(), _s(stream)), "moe_debug_grouped_down")
 
 
 def moe_layer_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> int:

@@ -382,6 +382,47 @@ int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* stream)
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_encode");
 }
 
+int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales, int64_t T, int H, int top_k,
+                           const float* topk_w, const int32_t* expert_offsets, const int32_t* sorted_pairs, int E,
+                           int I, const uint8_t* w_down, const float* s_down, float* y, void* ws, size_t ws_bytes,
+                           void* stream)
+{
+    if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOP_K) return MOE_ERR_INVALID_ARG;
+    if (I < 1 || I > MOE_MAX_INTERMEDIATE) return MOE_ERR_INVALID_ARG;
+    if (I % 16 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T * top_k > (int64_t(1) << 31) - 1) return MOE_ERR_UNSUPPORTED;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!h_codes || !h_scales || !topk_w || !expert_offsets || !sorted_pairs || !w_down || !s_down || !y))
+        return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {h_codes, h_scales, topk_w, expert_offsets, sorted_pairs, w_down, s_down, y, ws};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    if (int r = check_device()) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int r = clear_status(ws, s)) return r;
+    if (T == 0) return MOE_OK;
+    FfnArgs a{};
+    a.T = T;
+    a.H = H;
+    a.topk_w = topk_w;
+    a.k = top_k;
+    a.expert_offsets = expert_offsets;
+    a.sorted_pairs = sorted_pairs;
+    a.E = E;
+    a.I = I;
+    a.w_down = w_down;
+    a.s_down = s_down;
+    a.y = y;
+    a.status = static_cast<int*>(ws);
+    a.h_codes = const_cast<uint8_t*>(h_codes);
+    a.h_scales = const_cast<float*>(h_scales);
+    a.down_only = 1;
+    cudaError_t err = launch_grouped_ffn(a, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_grouped_down");
+}
+
 int moe_ffn_intermediate(const void* ws, int64_t T, int H, int I, int top_k, const uint8_t** h_codes,
                          const float** h_scales)
 {

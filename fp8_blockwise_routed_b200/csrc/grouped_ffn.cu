@@ -834,7 +834,8 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     cudaError_t err = stage_mark(a, 0, s);
     if (err != cudaSuccess) return err;
     // 1. gather the A operand rows (and their scales) into expert order
-    {
+    // (down_only: the caller supplies the intermediate; steps 1 and 3 are skipped)
+    if (!a.down_only) {
         const int64_t want = ceil_div64(P, 8);
         const int64_t cap = static_cast<int64_t>(di.sm_count) * 16;
         gather_rows_kernel<<<static_cast<int>(want < cap ? want : cap), 256, 0, s>>>(
@@ -855,9 +856,10 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
         const uint64_t sH[1] = {static_cast<uint64_t>(Ip)};
         const uint64_t dD[3] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H), static_cast<uint64_t>(E)};
         const uint64_t sD[2] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H) * I};
-        if (!make_tmap(&tmA1, a.a_sorted, 2, dA, sA, 128) || !make_tmap(&tmG, a.w_gate, 3, dW, sW, 128) ||
-            !make_tmap(&tmU, a.w_up, 3, dW, sW, 128) || !make_tmap(&tmA2, a.h_codes, 2, dH, sH, 128) ||
-            !make_tmap(&tmD, a.w_down, 3, dD, sD, 128))
+        if (!a.down_only && (!make_tmap(&tmA1, a.a_sorted, 2, dA, sA, 128) ||
+                             !make_tmap(&tmG, a.w_gate, 3, dW, sW, 128) || !make_tmap(&tmU, a.w_up, 3, dW, sW, 128)))
+            return cudaErrorNotSupported;
+        if (!make_tmap(&tmA2, a.h_codes, 2, dH, sH, 128) || !make_tmap(&tmD, a.w_down, 3, dD, sD, 128))
             return cudaErrorNotSupported;
     }
     const int grid = di.sm_count;
@@ -886,8 +888,10 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     g.H = H;
     g.status = a.status;
     if ((err = stage_mark(a, 1, s)) != cudaSuccess) return err;
-    err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
-    if (err != cudaSuccess) return err;
+    if (!a.down_only) {
+        err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
+        if (err != cudaSuccess) return err;
+    }
 
     // 4. down GEMM with the routing-weighted row epilogue
     GemmParams d = g;

@@ -127,6 +127,9 @@ struct FfnArgs {
     uint16_t* out_bf16;    // nullable
     int* cnt;              // workspace: arrival counters
     int32_t* nvalid;       // workspace: valid slots per token
+    // test hook: h_codes / h_scales are caller-supplied and only the down
+    // GEMM runs (no gather, no gate/up)
+    int down_only;
 };
 size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
                             size_t* off_sh, size_t* off_cnt = nullptr, size_t* off_nv = nullptr);

@@ -173,9 +173,12 @@ MOE_API int moe_route_quant(const float* logits, const uint16_t* x, int64_t T, i
  *     T*top_k*4 bytes plus alignment (T = 16384, E = 1024, top_k = 8 fits).
  *     Larger requests return MOE_ERR_WORKSPACE before anything is enqueued;
  *     moe_route_noalloc_error() then names the sizes.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture on the device.
+ *   - The first call in a CUDA context looks up the array's device address
+ *     (cudaGetSymbolAddress) with that context current, and caches it with
+ *     the context's id; a later call from another context (for instance
+ *     after cudaDeviceReset created a new one) looks it up again.  Make the
+ *     first call in a context before any stream capture in it.
+ *   - T is capped as for moe_route (MOE_ERR_UNSUPPORTED beyond it).
  *   - All calls share the one array: calls whose kernels overlap on the GPU
  *     (other streams, other host threads) race with each other.  Serialise
  *     them, e.g. on one stream.
@@ -282,7 +285,10 @@ MOE_API int moe_combine(const float* y, const int32_t* topk_ids, int64_t T, int 
 
 /* ---------------------------------------------------------------------------
  * moe_grouped_ffn_combine -- moe_grouped_ffn with moe_combine fused into the
- * down GEMM's epilogue (the plan's first "next" step).  Arguments as
+ * down GEMM's epilogue, so the routed FP32 rows are summed where they are
+ * written ("GLM-5.3-Flash EXL3 on CUDA ...", commit text: routed FP32 rows
+ * written in place, plan -> grouped gate/up -> grouped down -> combine).
+ * Arguments as
  * moe_grouped_ffn (y is still written: it carries the slot rows between the
  * GEMM's tiles) plus routed_scaling, out_f32 [T, H] and out_bf16 (nullable) as
  * moe_combine.  The down items run n-tile-major, so a token's k slot rows of
@@ -331,7 +337,8 @@ MOE_API int moe_combine_shared(const float* y, const int32_t* topk_ids, int64_t 
                                void* stream);
 
 /* ---------------------------------------------------------------------------
- * Expert parallelism across `world` GPUs ("next" row of the plan; reading:
+ * Expert parallelism across `world` GPUs.  The pages describe only
+ * single-GPU and tensor-parallel layers; the reading taken here is that
  * the layer shards by expert with one exchange on each side, and each
  * token's k slot rows are summed on its home GPU in slot order, so a row's
  * bits do not depend on the sharding -- "GLM-5.3-Flash EXL3 on CUDA ...",
@@ -465,6 +472,22 @@ MOE_API int moe_debug_encode(const float* in, int64_t n, uint8_t* out, void* str
  * arithmetic only; nothing is read from the device. */
 MOE_API int moe_ffn_intermediate(const void* ws, int64_t T, int H, int I, int top_k,
                                  const uint8_t** h_codes, const float** h_scales);
+
+/* moe_debug_grouped_down: the down GEMM of moe_grouped_ffn alone, on an
+ * intermediate the caller supplies: h_codes [T*top_k, Ip] uint8 E4M3 and
+ * h_scales [T*top_k, ceil(I/128)] FP32, rows in expert order (row r belongs
+ * to pair sorted_pairs[r]; rows at and beyond expert_offsets[E] are not
+ * read).  Writes y [T, top_k, H] FP32 for the valid pairs exactly as
+ * moe_grouped_ffn's down stage does (same kernel, same tiles).  It lets a
+ * test feed one and the same intermediate to this path and to an
+ * independent implementation, and so check the down projection and the
+ * combine without the requantisation decisions of the gate/up stage.
+ * Workspace: at least moe_combine_workspace_bytes() (the status word).
+ * Limits and errors as moe_grouped_ffn. */
+MOE_API int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales, int64_t T, int H, int top_k,
+                                   const float* topk_w, const int32_t* expert_offsets, const int32_t* sorted_pairs,
+                                   int E, int I, const uint8_t* w_down, const float* s_down, float* y, void* ws,
+                                   size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

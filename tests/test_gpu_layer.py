@@ -9,7 +9,8 @@ import torch
 
 import fp8_blockwise_routed_b200 as fm
 import moe_inputs as mi
-from gpu_helpers import assert_close_rows, check_layer, inputs, oracle_layer, run_layer, sha, tok_rel
+from gpu_helpers import (assert_close_rows, check_down_on_oracle_intermediate, check_layer, inputs, oracle_layer,
+                         oracle_layer_h, run_layer, sha, tok_rel)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +39,7 @@ def test_layer_small_every_element(name):
     d, h = inputs(wl)
     layer, out, _ = run_layer(wl, d)
     assert layer.device_status() == 0
-    ref = oracle_layer(wl, h, want_h=True)
+    ref = oracle_layer_h(wl, h)
     assert np.array_equal(layer.ids[: wl.T].cpu().numpy(), ref["ids"])
     assert np.array_equal(layer.codes[: wl.T].cpu().numpy(), ref["codes"])
     st = check_layer(wl, layer, out, ref, h)
@@ -53,10 +54,14 @@ def test_layer_workload_every_element(name):
     d, h = inputs(wl)
     layer, out, _ = run_layer(wl, d)
     assert layer.device_status() == 0
-    ref = oracle_layer(wl, h, want_h=True)
+    ref = oracle_layer_h(wl, h)
     st = check_layer(wl, layer, out, ref, h)
     print(name, st)
     assert st["flip_rate"] < 1e-3
+
+
+def _sampled(wl, layer):
+    return mi.sample_tokens(wl, layer.ids[: wl.T].cpu()).numpy()
 
 
 @pytest.mark.parametrize("name", ["glm", "long"])
@@ -69,12 +74,31 @@ def test_layer_workload_sampled(name):
     layer, out, _ = run_layer(wl, d)
     assert layer.device_status() == 0
     ids = layer.ids[: wl.T].cpu()
-    toks = mi.sample_tokens(wl, ids).numpy()
-    ref = oracle_layer(wl, h, tokens=toks, want_h=True)
+    toks = _sampled(wl, layer)
+    ref = oracle_layer_h(wl, h, tokens=toks)
     assert np.array_equal(ids.numpy(), ref["ids"])
     st = check_layer(wl, layer, out, dict(ref, ids=ref["ids"][toks], w=ref["w"][toks]), h, tokens=toks)
     print(name, len(toks), st)
     assert st["flip_rate"] < 1e-3
+
+
+@pytest.mark.parametrize("name", list(SMALL) + ["small", "non128", "glm", "long"])
+def test_down_and_combine_on_oracle_intermediate(name):
+    """Diagnostic of the down GEMM and the combine alone: the oracle's own
+    intermediate codes and scales go into the CUDA down GEMM (a test hook)
+    and the CUDA combine, so no requantisation decision can differ; every
+    compared output must meet the method's literal tolerance
+    |err| <= 2e-3 * ||row||_inf + 1e-3 with no allowance.  Full-size
+    workloads compare the oracle's token sample."""
+    wl = SMALL.get(name) or mi.WORKLOADS[name]
+    d, h = inputs(wl)
+    layer, out, _ = run_layer(wl, d)
+    assert layer.device_status() == 0
+    toks = _sampled(wl, layer) if name in ("glm", "long") else None
+    ref = oracle_layer_h(wl, h, tokens=toks)
+    assert np.array_equal(layer.ids[: wl.T].cpu().numpy(), ref["ids"])
+    st = check_down_on_oracle_intermediate(wl, layer, ref, h, tokens=toks)
+    print(name, st)
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiles", "h640"])
@@ -94,6 +118,35 @@ def test_row_invariance(name):
     for t in sorted({0, 1, wl.T // 2, wl.T - 1}):
         dd = dict(d, x=d["x"][t:t + 1].contiguous(), logits=d["logits"][t:t + 1].contiguous())
         assert torch.equal(run_layer(wl, dd)[1][0], full[t])
+
+
+@pytest.mark.parametrize("name", ["glm", "non128", "long"])
+def test_row_invariance_full_widths(name):
+    """Row invariance at the full workloads' widths (GEMM tiling, zero-padded
+    intermediate, K-block counts of the real shapes): sampled rows run alone
+    give the bits of the same rows in the full call (the first, middle and
+    last token, outlier tokens, a token of the least-loaded expert); the long
+    prefill also as four 4,096-row calls against the one 16,384-row call."""
+    wl = mi.WORKLOADS[name]
+    d, _ = inputs(wl)
+    layer, full, _ = run_layer(wl, d)
+    full = full.clone()
+    ids = layer.ids[: wl.T].cpu().numpy()
+    del layer
+    rows = {0, wl.T // 2, wl.T - 1}
+    if wl.x_dist == "normal_outliers":
+        rows |= set(mi.outlier_tokens(wl, 0).tolist()[:2])
+    counts = np.bincount(ids[ids >= 0].ravel(), minlength=wl.E)
+    active = np.nonzero(counts)[0]
+    least = active[np.argmin(counts[active])]
+    rows.add(int(np.nonzero((ids == least).any(axis=1))[0][0]))
+    for t in sorted(rows):
+        dd = dict(d, x=d["x"][t:t + 1].contiguous(), logits=d["logits"][t:t + 1].contiguous())
+        assert torch.equal(run_layer(wl, dd)[1][0], full[t]), f"row {t}"
+    if wl.T > 4096:
+        for t0 in range(0, wl.T, 4096):
+            dd = dict(d, x=d["x"][t0:t0 + 4096].contiguous(), logits=d["logits"][t0:t0 + 4096].contiguous())
+            assert torch.equal(run_layer(wl, dd)[1], full[t0:t0 + 4096]), f"rows {t0}..{t0 + 4095}"
 
 
 def test_row_invariance_4096_tiles():
