@@ -94,15 +94,24 @@ class ExpertParallelMoE:
         self.ws_ep = torch.empty((moe_ep_plan_workspace_bytes(T, k, world),), dtype=u8, device=dev)
         self.ws_ffn = torch.empty((moe_ffn_workspace_bytes(T, H, self.I, self.E_local, k),), dtype=u8, device=dev)
         self.ws_comb = torch.empty((moe_combine_workspace_bytes(),), dtype=u8, device=dev)
+        # the (owner, home) count tables are copied into pinned host memory
+        # as soon as the plan kernel has written them; the host waits for
+        # that copy (an event), not for the grouped FFN enqueued behind it
+        pin = dev.type == "cuda"
+        self._oh_h = torch.empty((world * world + 1,), dtype=i32, pin_memory=pin)
+        self._ho_h = torch.empty((world * world + 1,), dtype=i32, pin_memory=pin)
+        self._counts_ready = torch.cuda.Event() if pin else None
 
-    def counts(self, T: int):
-        """Rows this rank sends to each home and receives from each owner."""
+    def _split(self, oh, ho):
         w, r = self.world, self.rank
-        oh = self.offs_oh.cpu().tolist()
-        ho = self.offs_ho.cpu().tolist()
         send = [oh[r * w + h + 1] - oh[r * w + h] for h in range(w)]
         recv = [ho[r * w + o + 1] - ho[r * w + o] for o in range(w)]
         return send, recv
+
+    def counts(self, T: int):
+        """Rows this rank sends to each home and receives from each owner
+        (synchronous read of the device tables)."""
+        return self._split(self.offs_oh.cpu().tolist(), self.offs_ho.cpu().tolist())
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, stream=None) -> torch.Tensor:
         T = x.shape[0]
@@ -115,12 +124,23 @@ class ExpertParallelMoE:
         moe_route_quant(logits, x, k, ids, tw, self.offsets, self.sorted[:T * k], codes, scales, self.ws_route, stream)
         moe_ep_plan(ids, self.E, w, r, T_home, local_ids, self.send_rows[:T * k], recv_rows, self.offs_oh,
                     self.offs_ho, self.ws_ep, stream)
+        if self._counts_ready is not None:
+            s = torch.cuda.current_stream() if stream is None else stream
+            with torch.cuda.stream(s):
+                self._oh_h.copy_(self.offs_oh, non_blocking=True)
+                self._ho_h.copy_(self.offs_ho, non_blocking=True)
+            self._counts_ready.record(s)
         moe_permute(local_ids, self.E_local, self.offsets_local, self.sorted_local[:T * k], self.ws_perm, stream)
-        # the send buffer has a row for every pair, so the grouped FFN is
-        # enqueued before the counts reach the host
+        # The send buffer has a row for every pair (T*k rows, whatever this
+        # rank's share turns out to be), so the grouped FFN is enqueued before
+        # the counts reach the host and runs while the host reads them.
         moe_grouped_ffn_rows(codes, scales, local_ids, tw, self.offsets_local, self.sorted_local[:T * k], *self.w,
                              self.send[:T * k], self.send_rows[:T * k], self.ws_ffn, stream)
-        send_counts, recv_counts = self.counts(T)
+        if self._counts_ready is not None:
+            self._counts_ready.synchronize()  # routing and plan done; the FFN may still run
+            send_counts, recv_counts = self._split(self._oh_h.tolist(), self._ho_h.tolist())
+        else:
+            send_counts, recv_counts = self.counts(T)
         exchange_rows(self.send, send_counts, self.recv, recv_counts, self.group)
         out = self.out[:t1 - t0]
         moe_combine_rows(self.recv[:max(sum(recv_counts), 1)], recv_rows[:t1 - t0], self.rs, out, None,

@@ -104,3 +104,22 @@ def test_ep_plan_rejects_bad_arguments():
         fm.moe_ep_plan(ids, 8, 3, 0, 3, z, z, z, z, z, ws)
     with pytest.raises(fm.MoeError):  # homes do not cover the tokens
         fm.moe_ep_plan(ids, 9, 3, 0, 2, z, z, z, z, z, ws)
+
+
+def test_expert_parallel_against_oracle():
+    """Two emulated ranks on the tiny workload, compared with the oracle at the
+    method's tolerance (the other tests compare with the single-GPU layer bit
+    for bit); tokens the oracle routes nowhere are exact zeros."""
+    import numpy as np
+
+    import oracle
+    from gpu_helpers import assert_close_rows
+
+    wl = mi.WORKLOADS["tiny"]
+    d = mi.make_inputs(wl, 0, "cuda")
+    h = {k: v.cpu() for k, v in d.items()}
+    ref = oracle.moe_layer(h["x"], h["logits"], wl.k, h["w_gate"], h["s_gate"], h["w_up"], h["s_up"], h["w_down"],
+                           h["s_down"], wl.routed_scaling)
+    got = _emulate(wl, d, 2)
+    assert_close_rows(got, ref["out"])
+    assert np.all(ref["out"][np.all(ref["ids"] < 0, axis=1)] == 0)
