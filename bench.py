@@ -193,9 +193,10 @@ def gateup_alg_bytes(wl, active: int, P: int) -> float:
             + wl.T * wl.H + 4.0 * wl.T * wl.GH + P * wl.Ip + 4.0 * P * wl.GI)
 
 
-def cpu_baseline(wl, d, budget_tokens: int | None = None):
+def cpu_baseline(wl, d, budget_tokens: int | None = None, seconds: float = 20.0):
     """The oracle as it stands (plain C, FP64, OpenMP) on a seeded token
-    sample of the same workload, timed on the host.  Returns tokens/s."""
+    sample of the same workload (sized to about ``seconds`` of work), timed
+    on the host.  Returns tokens/s."""
     import oracle
 
     g = mi.generator(0, "cpu_baseline", "cpu")
@@ -212,9 +213,9 @@ def cpu_baseline(wl, d, budget_tokens: int | None = None):
 
     if budget_tokens:
         n = budget_tokens
-    else:  # size the sample to 10-20 s of oracle work (a 16-token probe underestimates the rate)
+    else:  # size the sample to the requested oracle work (a 16-token probe underestimates the rate)
         probe = min(16, wl.T)
-        n = max(probe, min(wl.T, int(20.0 * probe / max(run(probe), 1e-6))))
+        n = max(probe, min(wl.T, int(seconds * probe / max(run(probe), 1e-6))))
     dt = run(n)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n} seeded tokens of the {wl.name} workload (quantise, route, FFN, combine), "
@@ -310,6 +311,92 @@ class E2EPipeline:
         return t0.elapsed_time(t1)
 
 
+def gemm_roofline_s(wl, P: int, active: int, pk) -> float:
+    """max(FLOPs / FP8 peak, weight and scale bytes / HBM) of the two grouped
+    GEMMs (real I, valid pairs, active experts' weights once)."""
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal FP8:BF16 ratio 2 on the measured BF16 peak
+    wbytes = mi.algorithmic_bytes(wl, active) - wl.T * wl.H * 4 - wl.T * wl.H * 2 - wl.T * wl.E * 4
+    return max(mi.flops_per_layer(wl, P) / (fp8_peak * 1e12), wbytes / (pk["hbm_gbs"] * 1e9))
+
+
+def measure_workload(wl, steps: int, warmup: int, seed: int, pk, with_cpu: bool):
+    """One workload through the graph-launched layer: device time per step
+    over `steps` replays, per-stage means from the graph's event nodes, the
+    grouped GEMMs against their roofline, and the oracle on a ~3 s token
+    sample of the same inputs."""
+    import fp8_blockwise_routed_b200 as fm
+
+    d = mi.make_inputs(wl, seed=seed, device="cuda")
+    x_in = d["x"].clone()
+    lg_in = d["logits"].clone()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    plan = fm.LayerPlan(x_in, lg_in, wl.k, d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"],
+                        d["s_down"], wl.routed_scaling, stage_events=ev)
+    for _ in range(warmup):
+        plan.launch()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for _ in range(steps):
+        plan.launch()
+    t1.record(s)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    spans = {"route_quant": (0, 1), "gather": (1, 2), "gemm_gateup": (2, 3), "gemm_down": (3, 4),
+             "combine": (4, 5)}
+    acc = {n: [] for n in spans}
+    for _ in range(max(steps, 5)):
+        plan.launch()
+        torch.cuda.synchronize()
+        for n, (a, b) in spans.items():
+            acc[n].append(ev[a].elapsed_time(ev[b]))
+    st = {n: statistics.mean(v) for n, v in acc.items()}
+    status = plan.device_status()
+    ws = plan.ws
+    T, H, I, E, k = plan.shape
+    # expert offsets live in the plan's workspace; the layer's own view gives them
+    layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"], wl.k,
+                         wl.routed_scaling, wl.T)
+    layer.forward(d["x"], d["logits"])
+    torch.cuda.synchronize()
+    off = layer.offsets.cpu()
+    P = int(off[-1])
+    active = int(((off[1:] - off[:-1]) > 0).sum())
+    gemm_s = (st["gemm_gateup"] + st["gemm_down"]) / 1e3
+    flops = mi.flops_per_layer(wl, P)
+    roof = gemm_roofline_s(wl, P, active, pk)
+    res = {"ms_per_step": ms, "tokens_per_s": wl.T / (ms / 1e3), "stages_ms": st,
+           "gemm_tflops": flops / gemm_s / 1e12, "gemm_roofline_ms": roof * 1e3,
+           "gemm_frac_roofline": roof / gemm_s, "pairs": P, "active_experts": active,
+           "device_status": status | layer.device_status()}
+    if with_cpu:
+        res["cpu_oracle"] = cpu_baseline(wl, d, seconds=3.0)
+    plan.close()
+    del plan, layer, d, x_in, lg_in, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def layer_only(wl, n: int):
+    """The layer of `wl` (seed 0) n times through moe_route_quant,
+    moe_grouped_ffn and moe_combine, for profiler captures: each call launches
+    route_topk, route_rank, route_scatter, gather_rows, grouped_gemm (gate/up),
+    grouped_gemm (down) and combine, in that order."""
+    import fp8_blockwise_routed_b200 as fm
+
+    d = mi.make_inputs(wl, seed=0, device="cuda")
+    layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"], wl.k,
+                         wl.routed_scaling, wl.T)
+    for _ in range(n):
+        layer.forward(d["x"], d["logits"])
+    torch.cuda.synchronize()
+    off = layer.offsets.cpu()
+    print(json.dumps({"workload": wl.name, "calls": n, "device_status": layer.device_status(),
+                      "pairs": int(off[-1]), "active_experts": int(((off[1:] - off[:-1]) > 0).sum())}))
+
+
 def workload_config(wl):
     return {"workload": f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} top_k={wl.k} I={wl.I} "
                         f"rs={wl.routed_scaling} x={wl.x_dist} logits={wl.logit_dist}",
@@ -325,9 +412,17 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--workload", default="glm", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload lines of the other configurations")
+    ap.add_argument("--layer-only", type=int, default=0, metavar="N",
+                    help="run the workload's layer N times through the separate calls and exit "
+                         "(the program profiler captures run)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = mi.WORKLOADS[args.workload]
+    if args.layer_only:
+        layer_only(wl, args.layer_only)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
         return
@@ -418,9 +513,7 @@ def main():
     flops = mi.flops_per_layer(wl, P)
     gemm_s = (stage_ms["gemm_gateup"] + stage_ms["gemm_down"]) / 1e3
     fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal FP8:BF16 ratio 2 on the measured BF16 peak
-    layer_bytes = mi.algorithmic_bytes(wl, active)
-    roof_s = max(flops / (fp8_peak * 1e12), (layer_bytes - wl.T * wl.H * 4 - wl.T * wl.H * 2 - wl.T * wl.E * 4)
-                 / (pk["hbm_gbs"] * 1e9))
+    roof_s = gemm_roofline_s(wl, P, active, pk)
     traffic = recorded_traffic(f"gemm_gateup/{wl.name}")
 
     # end to end through the C ABI with host buffers
@@ -465,6 +558,19 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, d)
 
+    # every other workload on this rank's GPU, one after the other (the
+    # headline's buffers released first)
+    configs = {}
+    if not args.no_configs:
+        plan2.close()
+        del pipe, plan2, x_in2, lg_in2
+        torch.cuda.empty_cache()
+        for name in ("tiny", "small", "non128", "long"):
+            if name == wl.name:
+                continue
+            configs[name] = measure_workload(mi.WORKLOADS[name], args.steps, args.warmup, rank_seed(rank), pk,
+                                             with_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -506,9 +612,18 @@ def main():
             line["cpu_baseline"] = cpu
         if clocks:
             line["clocks"] = clocks
+        if configs:
+            configs[wl.name] = {"ms_per_step": ms_step, "tokens_per_s": wl.T / (ms_step / 1e3),
+                                "stages_ms": stage_ms, "gemm_tflops": flops / gemm_s / 1e12,
+                                "gemm_roofline_ms": roof_s * 1e3, "gemm_frac_roofline": roof_s / gemm_s,
+                                "pairs": P, "active_experts": active, "device_status": status}
+            if cpu:
+                configs[wl.name]["cpu_oracle"] = cpu
+            line["configs"] = configs
         print(json.dumps(line), flush=True)
     plan.close()
-    plan2.close()
+    if args.no_configs:
+        plan2.close()
     if world > 1:
         torch.distributed.destroy_process_group()
 

@@ -76,6 +76,9 @@ WORKLOADS = {
     # GLM widths with 64 experts (1.5 GB of weights): the case detailed
     # profiler captures run on (larger than L2, a few GB on the device)
     "glm64": Workload("glm64", 2048, 5120, 64, 8, 1536, 1.0, "normal_outliers", "zipf"),
+    # the long prefill's widths and rows with 32 experts (1.2 GB of weights):
+    # the case its DRAM traffic is captured on, scaled to the full layer
+    "long32": Workload("long32", 16384, 6144, 32, 8, 2048, 1.0, "student_t3", "zipf"),
 }
 
 
