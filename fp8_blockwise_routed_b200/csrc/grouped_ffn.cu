@@ -191,6 +191,12 @@ __device__ __forceinline__ Item decode_item(const int* seg, const int* ipre, int
     return it;
 }
 
+// A gate/up tile whose valid rows fit in 64: it takes the M = 64 path.
+__device__ __forceinline__ bool small_tile(const int* seg, const Item& w)
+{
+    return seg[w.e + 1] - (seg[w.e] + w.mt * BM) <= 64;
+}
+
 // ---------------------------------------------------------------- roles
 
 // Weight producer (one lane): the two 128-row weight boxes of every K block
@@ -265,15 +271,22 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
 // block is promoted with its own scales), then commits that free the A and B
 // stages and hand the buffer to the epilogue.  A commit tracks the MMAs of
 // the issuing thread only, which are exactly the ones it hands over.
+// Gate/up tiles with at most 64 valid rows use M = 64 MMAs (the accumulator
+// then sits in lanes 0-15 of each 32-lane quarter), which halves the
+// promotion work of their epilogue.
 template <int MODE>
-__device__ __forceinline__ void mma_role(const GemmParams& p, int total_items, uint32_t sbase, uint32_t bars,
-                                         uint32_t tmem, volatile int* abort, int parity)
+__device__ __forceinline__ void mma_role(const GemmParams& p, const int* seg, const int* ipre, int total_items,
+                                         uint32_t sbase, uint32_t bars, uint32_t tmem, volatile int* abort,
+                                         int parity)
 {
     constexpr int BS = b_stages<MODE>();
-    constexpr uint32_t idesc = idesc_e4m3_f32(128, 256);
+    constexpr uint32_t idesc128 = idesc_e4m3_f32(128, 256);
+    constexpr uint32_t idesc64 = idesc_e4m3_f32(64, 256);
     int it = 0;
     int last_commit = -1;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        uint32_t idesc = idesc128;
+        if (MODE == 0 && small_tile(seg, decode_item<false>(seg, ipre, p.E, item, p.rev))) idesc = idesc64;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             if ((it & 1) != parity) continue;  // the other issuer's K block
             const int sa = it % A_STAGES, sb = it % BS, b = it & 1;
@@ -305,6 +318,70 @@ drain:
         volatile int no_abort = 0;
         mbar_wait_bounded(bars + 8 * (BAR_TFULL + (last_commit & 1)), (last_commit >> 1) & 1, &no_abort,
                           WAIT_NS / 4);
+    }
+}
+
+// Gate/up epilogue of an M = 64 tile (layout above): h = SiLU(g) * u, the
+// 1x128 group quantiser of each row (the row's 128 columns sit in 4 lanes of
+// this warp and 4 of the partner warp of the other column half), codes
+// stored two at a time.  Same arithmetic per value as the 128-row path.
+__device__ __forceinline__ void small_tail(const GemmParams& p, const Item& w, int q, int half, int lane, int gA,
+                                           int gB, int row_end, float (&acc0)[64], float (&acc1)[64],
+                                           float* amax_x, int nitem, uint32_t xbar0, volatile int* abort)
+{
+    float amA = 0.f, amB = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float g = acc0[i];
+        const float e = ex2_approx_ftz(-g * 1.4426950408889634f);
+        const float h = (g * rcp_approx_ftz(1.0f + e)) * acc1[i];
+        acc0[i] = h;
+        if (i & 2) amB = fmax_nan(amB, fabsf(h));
+        else amA = fmax_nan(amA, fabsf(h));
+    }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+        amA = fmax_nan(amA, __shfl_xor_sync(0xFFFFFFFFu, amA, off));
+        amB = fmax_nan(amB, __shfl_xor_sync(0xFFFFFFFFu, amB, off));
+    }
+    const int rA = 16 * q + (lane >> 2), rB = rA + 8;
+    const int par = nitem & 1;
+    if ((lane & 3) == 0) {
+        amax_x[(par * 2 + half) * 128 + rA] = amA;
+        amax_x[(par * 2 + half) * 128 + rB] = amB;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xbar0 + 8 * q);
+    if (!__all_sync(0xFFFFFFFFu, mbar_spin_bounded(xbar0 + 8 * q, static_cast<uint32_t>(nitem & 1), abort, WAIT_NS)))
+        return;
+    const float oA = amax_x[(par * 2 + (half ^ 1)) * 128 + rA];
+    const float oB = amax_x[(par * 2 + (half ^ 1)) * 128 + rB];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int grow = rr ? gB : gA;
+        if (grow >= row_end) continue;
+        const float am = rr ? amB : amA, ot = rr ? oB : oA;
+        const bool nonfinite = !isfinite(am) || !isfinite(ot);
+        float s = __fdiv_rn(fmaxf(am, ot), 448.0f);
+        if (s == 0.f) s = 1.f;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.h_codes + static_cast<int64_t>(grow) * p.Ip + w.nt * 128 +
+                                                    half * 64 + 2 * (lane & 3));
+        if (nonfinite) {
+            s = __int_as_float(0x7FC00000);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[4 * i] = 0x7F7F;
+        } else {
+            const float inv = __frcp_rn(s);
+            const bool div = !isfinite(inv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float x0 = acc0[4 * i + 2 * rr], x1 = acc0[4 * i + 2 * rr + 1];
+                const float q0 = div ? __fdiv_rn(x0, s) : x0 * inv;
+                const float q1 = div ? __fdiv_rn(x1, s) : x1 * inv;
+                dst[4 * i] = static_cast<uint16_t>(e4m3x2(q0, q1));
+            }
+        }
+        if (half == 0 && (lane & 3) == 0) p.h_scales[static_cast<int64_t>(grow) * p.GI + w.nt] = s;
     }
 }
 
@@ -357,6 +434,46 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
         for (int i = 0; i < 64; ++i) {
             acc0[i] = 0.f;
             acc1[i] = 0.f;
+        }
+        if (MODE == 0 && small_tile(seg, w)) {
+            // M = 64 tile: rows 16q + j/4 ... live in lanes 0-15 of quarter q.
+            // This thread holds rows rA = 16q + lane/4 and rB = rA + 8, 16
+            // gate and 16 up columns of each (its half's 64 columns, 2 per
+            // 8-column group): acc0[4i + e] / acc1[4i + e], e < 2 row rA,
+            // e >= 2 row rB, columns half*64 + 8i + 2(lane%4) + (e&1).
+            const int gA = seg[w.e] + w.mt * BM + 16 * q + (lane >> 2), gB = gA + 8;
+            const float* saA = p.a_scales + static_cast<int64_t>(gA < p.P ? gA : p.P - 1) * p.num_kb;
+            const float* saB = p.a_scales + static_cast<int64_t>(gB < p.P ? gB : p.P - 1) * p.num_kb;
+            const float* s0 = p.b_s0 + (static_cast<int64_t>(w.e) * p.b_nblocks + w.nt) * p.num_kb;
+            const float* s1 = p.b_s1 + (static_cast<int64_t>(w.e) * p.b_nblocks + w.nt) * p.num_kb;
+            float aA_n = __ldg(saA), aB_n = __ldg(saB), w0_n = __ldg(s0), w1_n = __ldg(s1);
+            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                const float c0A = aA_n * w0_n, c0B = aB_n * w0_n;
+                const float c1A = aA_n * w1_n, c1B = aB_n * w1_n;
+                if (kb + 1 < p.num_kb) {
+                    aA_n = __ldg(saA + kb + 1);
+                    aB_n = __ldg(saB + kb + 1);
+                    w0_n = __ldg(s0 + kb + 1);
+                    w1_n = __ldg(s1 + kb + 1);
+                }
+                const int b = it & 1;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, (it >> 1) & 1, abort, WAIT_NS)))
+                    return;
+                const uint32_t col = lane_base + b * 256 + half * 64;
+                uint32_t ra[32], rb[32];
+                tmem_ld16x256_x8_issue(col, ra);        // gate columns
+                tmem_ld_wait(ra);
+                tmem_ld16x256_x8_issue(col + 128, rb);  // up columns
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc0[i] = fmaf((i & 2) ? c0B : c0A, __uint_as_float(ra[i]), acc0[i]);
+                tmem_ld_wait(rb);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty0 + 8 * b);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc1[i] = fmaf((i & 2) ? c1B : c1A, __uint_as_float(rb[i]), acc1[i]);
+            }
+            small_tail(p, w, q, half, lane, gA, gB, seg[w.e + 1], acc0, acc1, amax_x, nitem, xbar0, abort);
+            continue;
         }
         // scales of K block kb+1 are fetched while block kb is promoted
         float sa_n = __ldg(sa_row), w0_n = __ldg(s0), w1_n = has1 ? __ldg(s1) : 0.f;
@@ -643,7 +760,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         setmaxnreg_dec<REGS_CTRL>();
         if ((threadIdx.x & 31) == 0) {
             if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
-            else if (warp == 1 || warp == 2) mma_role<MODE>(p, total_items, sbase, bars, tmem, abort, warp - 1);
+            else if (warp == 1 || warp == 2)
+                mma_role<MODE>(p, seg, ipre, total_items, sbase, bars, tmem, abort, warp - 1);
             else if (warp == 3) producer_a<MODE>(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {

@@ -249,6 +249,24 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32])
                  : "memory");
 }
 
+// 16 TMEM lanes x 64 consecutive FP32 columns (the .16x256b shape repeated
+// 8 times), issued into r; wait with tmem_ld_wait.  Thread t receives, for
+// repetition i (columns 8i .. 8i+7): r[4i], r[4i+1] = lane t/4, columns
+// 8i + 2(t%4) and +1; r[4i+2], r[4i+3] = lane t/4 + 8, the same columns.
+__device__ __forceinline__ void tmem_ld16x256_x8_issue(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored in the
 // 128-byte-swizzled canonical layout: rows of 128 bytes, 8-row atoms of
 // 1024 bytes stacked contiguously (stride-dimension offset 1024 B).
