@@ -194,6 +194,55 @@ def make_weights(wl: Workload, seed: int = 0, device="cpu", experts_per_chunk: i
     return out
 
 
+def _mx_fp8(W: torch.Tensor):
+    """W [n_e, R, C] FP32 (C % 32 == 0) -> MXFP8: codes uint8 [n_e,R,C] and
+    one UE8M0 scale byte per (row, 32 columns) [n_e,R,C/32]: shared exponent
+    floor(log2(amax)) - 8, element = float8_e4m3fn(W / 2^se) after clamping to
+    +-448.  Input preparation (the checkpoint format), not a step of the path."""
+    n_e, R, C = W.shape
+    blk = W.view(n_e, R, C // 32, 32)
+    amax = blk.abs().amax(dim=-1)
+    _, ex = torch.frexp(amax)
+    se = torch.where(amax == 0, torch.full_like(ex, -127), (ex - 9).clamp(-127, 127))
+    q = (blk * torch.ldexp(torch.ones_like(amax), -se)[..., None]).clamp(-FP8_MAX, FP8_MAX)
+    codes = q.to(torch.float8_e4m3fn).view(torch.uint8).view(n_e, R, C).contiguous()
+    return codes, (se + 127).to(torch.uint8).contiguous()
+
+
+def make_weights_mx(wl: Workload, seed: int = 0, device="cpu", experts_per_chunk: int | None = None):
+    """The weights of make_weights (the same FP32 draws) stored as MXFP8:
+    w_gate, w_up [E,I,H] u8 with s_gate, s_up [E,I,H/32] u8 (UE8M0);
+    w_down [E,H,I] u8 with s_down [E,H,I/32] u8."""
+    E, I, H = wl.E, wl.I, wl.H
+    assert I % 32 == 0 and H % 32 == 0
+    if experts_per_chunk is None:
+        experts_per_chunk = max(1, (1 << 27) // (I * H))
+    out = {}
+    for name, (R, C) in (("gate", (I, H)), ("up", (I, H)), ("down", (H, I))):
+        g = generator(seed, f"w_{name}", device)
+        codes = torch.empty((E, R, C), dtype=torch.uint8, device=device)
+        scales = torch.empty((E, R, C // 32), dtype=torch.uint8, device=device)
+        for e0 in range(0, E, experts_per_chunk):
+            e1 = min(E, e0 + experts_per_chunk)
+            W = torch.randn((e1 - e0, R, C), generator=g, device=device, dtype=torch.float32) * 0.02
+            c, sc = _mx_fp8(W)
+            codes[e0:e1] = c
+            scales[e0:e1] = sc
+            del W, c, sc
+        out[f"w_{name}"] = codes
+        out[f"s_{name}"] = scales
+    return out
+
+
+def make_inputs_mx(wl: Workload | str, seed: int = 0, device="cpu", T: int | None = None):
+    """All inputs of one MXFP8 layer call (x and logits as make_inputs)."""
+    if isinstance(wl, str):
+        wl = WORKLOADS[wl]
+    d = {"x": make_x(wl, seed, device, T), "logits": make_logits(wl, seed, device, T)}
+    d.update(make_weights_mx(wl, seed, device))
+    return d
+
+
 def make_inputs(wl: Workload | str, seed: int = 0, device="cpu", T: int | None = None):
     """All inputs of one layer call: x, logits, weights and scales."""
     if isinstance(wl, str):
@@ -238,6 +287,7 @@ def ceil_div(a: int, b: int) -> int:
     return -(-a // b)
 
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_x", "make_logits", "make_weights",
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_inputs_mx", "make_x", "make_logits", "make_weights",
+           "make_weights_mx",
            "outlier_tokens", "masked_experts", "sample_tokens", "flops_per_layer",
            "algorithmic_bytes", "generator", "ceil_div", "math"]

@@ -58,6 +58,12 @@ def open_library(path: str) -> ctypes.CDLL:
                                    P, P, P, P, P, P, ctypes.c_double,
                                    P, i64, P, P, P, P, P, P, P, i32]
     lib.oracle_num_threads.restype = i32
+    lib.oracle_ue8m0_decode.restype = ctypes.c_double
+    lib.oracle_ue8m0_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_mx_quant_block.argtypes = [P, i32, P, P]
+    lib.oracle_mx_quant_act.argtypes = [P, i64, i64, P, P]
+    lib.oracle_mx_moe_ffn.argtypes = [P, P, i64, i64, P, P, i32, i32, i64, P, P, P, P, P, P, ctypes.c_double,
+                                      P, i64, P, P, P, P, i32]
     return lib
 
 
@@ -275,5 +281,86 @@ def moe_layer(x_bf16, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down,
     off, sp = permute(ids, E)
     res = moe_ffn(codes, scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_down,
                   routed_scaling, tokens=tokens, **kw)
+    res.update(codes=codes, scales=scales, ids=ids, w=w, offsets=off, sorted_pairs=sp)
+    return res
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 variant: E4M3 elements with one UE8M0 (power-of-two) scale per 32
+# values along the contraction dimension.  The pages only name an MXFP8 MoE
+# runtime as not yet qualified ("Exact AVX2 FP8 arithmetic conversion avoids
+# costly LUT gathers", "Real-checkpoint measurements"); the rules M1-M3 in
+# oracle.c are readings that follow the OCP Microscaling Formats v1.0.
+
+def ue8m0_decode(x: int) -> float:
+    """UE8M0 byte -> 2^(x-127); 0xFF -> NaN (reading M1)."""
+    return float(_load().oracle_ue8m0_decode(int(x) & 0xFF))
+
+
+def mx_quant_block(x: np.ndarray):
+    """1..32 FP32 values -> (codes uint8[n], scale byte) by reading M2."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    assert 1 <= x.size <= 32
+    codes = np.zeros(x.size, np.uint8)
+    sc = np.zeros(1, np.uint8)
+    _load().oracle_mx_quant_block(_ptr(x), x.size, _ptr(codes), _ptr(sc))
+    return codes, int(sc[0])
+
+
+def mx_quant_act(x_bf16_bits):
+    """BF16 rows [T,H] -> codes uint8 [T,H], UE8M0 scales uint8 [T,H/32]."""
+    if hasattr(x_bf16_bits, "detach"):
+        import torch
+        x_bf16_bits = x_bf16_bits.detach().cpu().contiguous().view(torch.int16).numpy()
+    x = np.ascontiguousarray(x_bf16_bits).view(np.uint16)
+    T, H = x.shape
+    assert H % 32 == 0
+    codes = np.zeros((T, H), np.uint8)
+    scales = np.zeros((T, H // 32), np.uint8)
+    _load().oracle_mx_quant_act(_ptr(x), T, H, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mx_moe_ffn(codes, act_scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling: float,
+               tokens=None, want_h: bool = False, n_threads: int = 0):
+    """Expert FFN + combine of the MXFP8 variant (reading M3).  Scales are
+    UE8M0 bytes: activations [T,H/32], gate/up [E,I,H/32], down [E,H,I/32]."""
+    codes = _np(codes, np.uint8)
+    act_scales = _np(act_scales, np.uint8)
+    ids = _np(ids, np.int32)
+    w = np.ascontiguousarray(np.asarray(w, dtype=np.float64))
+    wg, wu, wd = _np(w_gate, np.uint8), _np(w_up, np.uint8), _np(w_down, np.uint8)
+    sg, su, sd = _np(s_gate, np.uint8), _np(s_up, np.uint8), _np(s_down, np.uint8)
+    T, H = codes.shape
+    k = ids.shape[1]
+    E, I, _ = wg.shape
+    assert I % 32 == 0 and sg.shape == (E, I, H // 32) and sd.shape == (E, H, I // 32)
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int64)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    n = tokens.size
+    out = np.zeros((n, H), np.float64)
+    hc = np.zeros((n, k, I), np.uint8) if want_h else None
+    hs = np.zeros((n, k, I // 32), np.uint8) if want_h else None
+    hf = np.zeros((n, k, I), np.float32) if want_h else None
+    _load().oracle_mx_moe_ffn(_ptr(codes), _ptr(act_scales), T, H, _ptr(ids), _ptr(w), k, E, I, _ptr(wg),
+                              _ptr(sg), _ptr(wu), _ptr(su), _ptr(wd), _ptr(sd), float(routed_scaling),
+                              _ptr(tokens), n, _ptr(out), _ptr(hc), _ptr(hs), _ptr(hf), int(n_threads))
+    res = {"out": out}
+    if want_h:
+        res["h_codes"], res["h_scales"], res["h_fp32"] = hc, hs, hf
+    return res
+
+
+def mx_moe_layer(x_bf16, logits, top_k, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling,
+                 tokens=None, **kw):
+    """The MXFP8 layer in the pages' order: quantise activations (M2), route,
+    permute, expert FFN (M3), combine."""
+    codes, scales = mx_quant_act(x_bf16)
+    ids, w = route(logits, top_k)
+    E = _np(w_gate, np.uint8).shape[0]
+    off, sp = permute(ids, E)
+    res = mx_moe_ffn(codes, scales, ids, w, w_gate, s_gate, w_up, s_up, w_down, s_down, routed_scaling,
+                     tokens=tokens, **kw)
     res.update(codes=codes, scales=scales, ids=ids, w=w, offsets=off, sorted_pairs=sp)
     return res

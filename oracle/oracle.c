@@ -77,11 +77,13 @@ ORACLE_API double oracle_e4m3_decode(uint8_t b)
 /* ------------------------------------------------------------------------ */
 /* E4M3 encode (reading R1): nearest finite code by explicit search.         */
 /* ------------------------------------------------------------------------ */
-ORACLE_API uint8_t oracle_e4m3_encode(float v)
+/* Nearest finite E4M3 code to an exact (double) value, ties to the code with
+ * an even mantissa LSB; magnitudes from 448 up (Inf included) saturate to the
+ * code of 448; the sign is kept for +-0. */
+static uint8_t e4m3_encode_exact(double v)
 {
-    if (isnan(v)) return 0x7F;
     int neg = signbit(v) ? 1 : 0;
-    double a = fabs((double)v);
+    double a = fabs(v);
     /* Saturation: every magnitude from the largest finite value (448) up to
      * and including Inf takes the code of 448. */
     if (a >= 448.0) return (uint8_t)(0x7E | (neg << 7));
@@ -97,6 +99,12 @@ ORACLE_API uint8_t oracle_e4m3_encode(float v)
         }
     }
     return (uint8_t)(best | (neg << 7));
+}
+
+ORACLE_API uint8_t oracle_e4m3_encode(float v)
+{
+    if (isnan(v)) return 0x7F;
+    return e4m3_encode_exact((double)v);  /* every FP32 value is exact in double */
 }
 
 /* Encode n values (tests sweep large sets of FP32 inputs through this). */
@@ -369,4 +377,151 @@ ORACLE_API int oracle_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ======================================================================== */
+/* MXFP8 variant (the pages name an MXFP8 MoE runtime as not yet qualified:   */
+/* [KT-2245] "Real-checkpoint measurements", caveats).  E4M3 elements with    */
+/* one UE8M0 (power-of-two) scale per 32 consecutive values along the         */
+/* contraction dimension.  Readings (the pages give no definition; these      */
+/* follow the OCP Microscaling Formats v1.0 rules):                           */
+/*   M1  UE8M0 byte X decodes to 2^(X-127); X = 0xFF is NaN.                  */
+/*   M2  Block quantiser over 32 values (fewer at a ragged end): amax =       */
+/*       max|x|; e = floor(log2(amax)); shared exponent se = e - 8 (8 is the  */
+/*       largest exponent of a normal E4M3 value, 448 = 1.75 * 2^8), clamped  */
+/*       to [-127, 127]; X = se + 127; code_i = the E4M3 code nearest to the  */
+/*       exact x_i / 2^se, ties to even, saturating at +-448.  amax = 0 ->    */
+/*       X = 0 and codes +-0; a block holding NaN or Inf -> X = 0xFF and      */
+/*       codes 0x7F.                                                          */
+/*   M3  The FFN is the blockwise path of oracle_moe_ffn with these scales:   */
+/*       activations and intermediate quantised by M2 per 32 columns,         */
+/*       weights stored with one UE8M0 scale per (row, 32 columns).           */
+/* ======================================================================== */
+
+/* M1 */
+ORACLE_API double oracle_ue8m0_decode(uint8_t x)
+{
+    if (x == 0xFF) return NAN;
+    return ldexp(1.0, (int)x - 127);
+}
+
+/* M2: n values (1..32) -> n codes and one scale byte. */
+ORACLE_API void oracle_mx_quant_block(const float* x, int n, uint8_t* codes, uint8_t* scale)
+{
+    int nonfinite = 0;
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        if (!isfinite(x[i])) nonfinite = 1;
+        else if (fabs((double)x[i]) > amax) amax = fabs((double)x[i]);
+    }
+    if (nonfinite) {
+        *scale = 0xFF;
+        for (int i = 0; i < n; ++i) codes[i] = 0x7F;
+        return;
+    }
+    int se;
+    if (amax == 0.0) {
+        se = -127;
+    } else {
+        int ex;
+        frexp(amax, &ex);      /* amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1 */
+        se = (ex - 1) - 8;
+        if (se < -127) se = -127;
+        if (se > 127) se = 127;
+    }
+    *scale = (uint8_t)(se + 127);
+    for (int i = 0; i < n; ++i) codes[i] = e4m3_encode_exact(ldexp((double)x[i], -se));
+}
+
+/* MX activation quantiser: x [T,H] BF16 bits -> codes [T,H], scales [T,H/32]. */
+ORACLE_API void oracle_mx_quant_act(const uint16_t* x, int64_t T, int64_t H, uint8_t* codes, uint8_t* scales)
+{
+    int64_t G = H / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float buf[32];
+        for (int64_t g = 0; g < G; ++g) {
+            for (int i = 0; i < 32; ++i) buf[i] = bf16_to_float(x[t * H + g * 32 + i]);
+            oracle_mx_quant_block(buf, 32, codes + t * H + g * 32, scales + t * G + g);
+        }
+    }
+}
+
+/* M3: expert FFN and combine with MX operands, for the tokens listed.
+ *   codes [T,H], act_scales [T,H/32] (UE8M0)          activations
+ *   ids [T,k], w [T,k] (FP64)                          routing
+ *   wg, wu [E,I,H]; sg, su [E,I,H/32] (UE8M0)           gate / up
+ *   wd [E,H,I];     sd [E,H,I/32]   (UE8M0)             down
+ *   out [n_tok,H] FP64; h_codes [n_tok,k,I], h_scales [n_tok,k,I/32],
+ *   h_fp32 [n_tok,k,I] (nullable).  I % 32 == 0. */
+ORACLE_API void oracle_mx_moe_ffn(const uint8_t* codes, const uint8_t* act_scales, int64_t T, int64_t H,
+                                  const int32_t* ids, const double* w, int k, int E, int64_t I,
+                                  const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,
+                                  const uint8_t* wd, const uint8_t* sd, double routed_scaling,
+                                  const int64_t* token_list, int64_t n_tok, double* out,
+                                  uint8_t* h_codes, uint8_t* h_scales, float* h_fp32, int n_threads)
+{
+    (void)T;
+    (void)E;
+    const int64_t BH = H / 32, BI = I / 32;
+    double dec[256], sdec[256];
+    for (int b = 0; b < 256; ++b) {
+        dec[b] = oracle_e4m3_decode((uint8_t)b);
+        sdec[b] = oracle_ue8m0_decode((uint8_t)b);
+    }
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel
+    {
+        double* xd = (double*)malloc((size_t)H * sizeof(double));
+        double* hd = (double*)malloc((size_t)I * sizeof(double));
+        float* h32 = (float*)malloc((size_t)I * sizeof(float));
+        uint8_t* hq = (uint8_t*)malloc((size_t)I);
+        uint8_t* sh = (uint8_t*)malloc((size_t)BI);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t it = 0; it < n_tok; ++it) {
+            int64_t t = token_list[it];
+            double* orow = out + it * H;
+            for (int64_t n = 0; n < H; ++n) orow[n] = 0.0;
+            for (int64_t kk = 0; kk < H; ++kk) xd[kk] = dec[codes[t * H + kk]] * sdec[act_scales[t * BH + kk / 32]];
+            for (int j = 0; j < k; ++j) {
+                int e = ids[t * k + j];
+                if (e < 0) continue;
+                const uint8_t* Wg = wg + (int64_t)e * I * H;
+                const uint8_t* Wu = wu + (int64_t)e * I * H;
+                const uint8_t* Sg = sg + (int64_t)e * I * BH;
+                const uint8_t* Su = su + (int64_t)e * I * BH;
+                for (int64_t n = 0; n < I; ++n) {
+                    double g = 0.0, u = 0.0;
+                    for (int64_t kk = 0; kk < H; ++kk) {
+                        g += xd[kk] * (dec[Wg[n * H + kk]] * sdec[Sg[n * BH + kk / 32]]);
+                        u += xd[kk] * (dec[Wu[n * H + kk]] * sdec[Su[n * BH + kk / 32]]);
+                    }
+                    h32[n] = (float)(g / (1.0 + exp(-g)) * u);
+                }
+                for (int64_t b = 0; b < BI; ++b) oracle_mx_quant_block(h32 + b * 32, 32, hq + b * 32, sh + b);
+                if (h_fp32) memcpy(h_fp32 + (it * k + j) * I, h32, (size_t)I * sizeof(float));
+                if (h_codes) memcpy(h_codes + (it * k + j) * I, hq, (size_t)I);
+                if (h_scales) memcpy(h_scales + (it * k + j) * BI, sh, (size_t)BI);
+                for (int64_t i = 0; i < I; ++i) hd[i] = dec[hq[i]] * sdec[sh[i / 32]];
+                const uint8_t* Wd = wd + (int64_t)e * H * I;
+                const uint8_t* Sd = sd + (int64_t)e * H * BI;
+                double wj = w[t * k + j];
+                for (int64_t n = 0; n < H; ++n) {
+                    double acc = 0.0;
+                    for (int64_t i = 0; i < I; ++i) acc += hd[i] * (dec[Wd[n * I + i]] * sdec[Sd[n * BI + i / 32]]);
+                    orow[n] += wj * acc;
+                }
+            }
+            for (int64_t n = 0; n < H; ++n) orow[n] *= routed_scaling;
+        }
+        free(xd);
+        free(hd);
+        free(h32);
+        free(hq);
+        free(sh);
+    }
 }

@@ -12,6 +12,7 @@ import pytest
 import oracle
 import test_oracle_codec as codec
 import test_oracle_ffn as ffn
+import test_oracle_mx as mx
 import test_oracle_route as route
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -31,17 +32,26 @@ MUTANTS = {
                          "sorted_pairs[offsets[e + 1] - 1 - (next[e]++ - offsets[e])] = (int32_t)p;"),
     "ffn_gate_scale_dropped": ("dec[Wg[n * H + kk]] * (double)Sg[(n / 128) * GH + kk / 128]", "dec[Wg[n * H + kk]]"),
     "ffn_act_scale_dropped": ("* (double)act_scales[t * GH + kk / 128]", "* 1.0"),
-    "ffn_silu_sign": ("g / (1.0 + exp(-g)) * u", "g / (1.0 + exp(g)) * u"),
+    "ffn_silu_sign": ("double h64 = g / (1.0 + exp(-g)) * u;", "double h64 = g / (1.0 + exp(g)) * u;"),
     "ffn_clamped_silu": ("double h64 = g / (1.0 + exp(-g)) * u;",
                          "double h64 = g / (1.0 + exp(-g)) * (u > 10 ? 10 : u < -10 ? -10 : u);"),
     "ffn_up_gate_swapped": ("* u;\n", "* g;\n"),
     "ffn_no_requant": ("for (int64_t i = 0; i < I; ++i) hd[i] = dec[hq_use[i]] * (double)sh_use[i / 128];",
                        "for (int64_t i = 0; i < I; ++i) hd[i] = h_override_codes ? dec[hq_use[i]] * (double)sh_use[i / 128] : (double)h32[i];"),
-    "ffn_down_transposed": ("dec[Wd[n * I + i]]", "dec[Wd[i * H + n]]"),
+    "ffn_down_transposed": ("acc += hd[i] * (dec[Wd[n * I + i]] * (double)", "acc += hd[i] * (dec[Wd[i * H + n]] * (double)"),
     "ffn_down_scale_index": ("Sd[(n / 128) * GI + i / 128]", "Sd[(n / 128) * GI]"),
     "ffn_routing_weight_dropped": ("orow[n] += wj * o[n];", "orow[n] += o[n];"),
-    "ffn_routed_scaling_dropped": ("orow[n] *= routed_scaling;", "orow[n] *= 1.0;"),
+    "ffn_routed_scaling_dropped": ("orow[n] *= routed_scaling;\n        }\n        free(xd);\n        free(o);",
+                                   "orow[n] *= 1.0;\n        }\n        free(xd);\n        free(o);"),
     "ffn_last_group_full_width": ("int64_t nc = (I - c0 < 128) ? (I - c0) : 128;", "int64_t nc = 128;"),
+    # the MXFP8 variant
+    "mx_ue8m0_bias": ("return ldexp(1.0, (int)x - 127);", "return ldexp(1.0, (int)x - 128);"),
+    "mx_shared_exponent_off_by_one": ("se = (ex - 1) - 8;", "se = (ex - 1) - 7;"),
+    "mx_weight_scale_dropped": ("g += xd[kk] * (dec[Wg[n * H + kk]] * sdec[Sg[n * BH + kk / 32]]);",
+                                "g += xd[kk] * (dec[Wg[n * H + kk]]);"),
+    "mx_block_of_64": ("sdec[act_scales[t * BH + kk / 32]]", "sdec[act_scales[t * BH + kk / 64]]"),
+    "mx_no_requant": ("hd[i] = dec[hq[i]] * sdec[sh[i / 32]];", "hd[i] = (double)h32[i];"),
+    "mx_zero_block_scale": ("if (amax == 0.0) {\n        se = -127;", "if (amax == 0.0) {\n        se = 0;"),
 }
 
 PINS = [
@@ -60,6 +70,11 @@ PINS = [
     (ffn.test_ffn_exact_integer_gate_up, ()),
     (ffn.test_ffn_invariants, ()),
     (ffn.test_ffn_nan_stays_in_its_row, ()),
+    (mx.test_ue8m0_decode_exhaustive, ()),
+    (mx.test_block_power_of_two_max, (3,)),
+    (mx.test_block_zero_and_nonfinite, ()),
+    (mx.test_block_vs_torch_restatement, ()),
+    (mx.test_mx_layer_vs_dense_bruteforce, ("tiny",)),
 ]
 
 
