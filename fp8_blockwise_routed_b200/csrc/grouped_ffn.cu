@@ -271,10 +271,11 @@ __device__ __forceinline__ void producer_a(const CUtensorMap* tmA, const GemmPar
 // block is promoted with its own scales), then commits that free the A and B
 // stages and hand the buffer to the epilogue.  A commit tracks the MMAs of
 // the issuing thread only, which are exactly the ones it hands over.
-// Gate/up tiles with at most 64 valid rows use M = 64 MMAs (the accumulator
-// then sits in lanes 0-15 of each 32-lane quarter), which halves the
-// promotion work of their epilogue.
-template <int MODE>
+// In the SMALL instantiation, tiles with at most 64 valid rows (gate/up and
+// down, not the fused combine) use M = 64 MMAs (the accumulator then sits in
+// lanes 0-15 of each 32-lane quarter), which halves the promotion work of
+// their epilogue.
+template <int MODE, bool SMALL>
 __device__ __forceinline__ void mma_role(const GemmParams& p, const int* seg, const int* ipre, int total_items,
                                          uint32_t sbase, uint32_t bars, uint32_t tmem, volatile int* abort,
                                          int parity)
@@ -286,7 +287,7 @@ __device__ __forceinline__ void mma_role(const GemmParams& p, const int* seg, co
     int last_commit = -1;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
         uint32_t idesc = idesc128;
-        if (MODE == 0 && small_tile(seg, decode_item<false>(seg, ipre, p.E, item, p.rev))) idesc = idesc64;
+        if (SMALL && MODE != 2 && small_tile(seg, decode_item<false>(seg, ipre, p.E, item, p.rev))) idesc = idesc64;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
             if ((it & 1) != parity) continue;  // the other issuer's K block
             const int sa = it % A_STAGES, sb = it % BS, b = it & 1;
@@ -385,7 +386,69 @@ __device__ __forceinline__ void small_tail(const GemmParams& p, const Item& w, i
     }
 }
 
-template <int MODE>
+// Down epilogue of an M = 64 tile (layout above): y[pair] = w_pair * o for
+// the thread's two rows.  The warp's 16 rows x 2 column segments (256 bytes
+// each) fill its 32 staging slots exactly, so each lane then sends one
+// segment by a bulk copy and no copy waits for another's read.
+__device__ __forceinline__ void small_down_tail(const GemmParams& p, const Item& w, int half, int lane, int gA,
+                                                int gB, int row_end, const float (&acc0)[64],
+                                                const float (&acc1)[64], uint32_t warp_slots)
+{
+    int yA = -1, yB = -1;
+    float wA = 0.f, wB = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int g = rr ? gB : gA;
+        if (g >= row_end) continue;
+        const int pair = __ldg(p.sorted_pairs + g);
+        int64_t yrow = -1;
+        float wt = 0.f;
+        if (pair >= 0 && pair < p.P) {
+            wt = __ldg(p.topk_w + pair);
+            yrow = p.y_rows ? __ldg(p.y_rows + pair) : pair;
+        }
+        if (pair < 0 || pair >= p.P || yrow >= p.y_nrows) {
+            atomicOr(p.status, kDevBadPair);
+            continue;
+        }
+        if (rr) {
+            yB = static_cast<int>(yrow);
+            wB = wt;
+        } else {
+            yA = static_cast<int>(yrow);
+            wA = wt;
+        }
+    }
+    // every slot of this warp has been read by the copies sent from it before
+    bulk_wait_read_all();
+    __syncwarp();
+    const int rA = lane >> 2, rB = rA + 8;  // rows within the warp's 16
+#pragma unroll
+    for (int sgm = 0; sgm < 2; ++sgm) {
+        const float* a = sgm ? acc1 : acc0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t off = (8 * i + 2 * (lane & 3)) * 4;
+            st_shared_v2(warp_slots + (sgm * 16 + rA) * STAGE_SLOT + off, wA * a[4 * i], wA * a[4 * i + 1]);
+            st_shared_v2(warp_slots + (sgm * 16 + rB) * STAGE_SLOT + off, wB * a[4 * i + 2], wB * a[4 * i + 3]);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    // lane L sends segment L/16 of row L%16; that row's y row comes from the
+    // lane holding it (4 * (row % 8), its first or second row)
+    const int sgm = lane >> 4, row = lane & 15;
+    const int src = 4 * (row & 7);
+    const int ya = __shfl_sync(0xFFFFFFFFu, yA, src);
+    const int yb = __shfl_sync(0xFFFFFFFFu, yB, src);
+    const int yrow = row < 8 ? ya : yb;
+    const int c = w.nt * 256 + sgm * 128 + half * 64;
+    if (yrow >= 0 && c < p.H)
+        bulk_store(p.y + static_cast<int64_t>(yrow) * p.H + c, warp_slots + (sgm * 16 + row) * STAGE_SLOT, 256);
+    bulk_commit();
+}
+
+template <int MODE, bool SMALL>
 __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* seg, const int* ipre, int total_items, uint32_t bars,
                               uint32_t tmem, float* amax_x, volatile int* abort)
 {
@@ -435,18 +498,21 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
             acc0[i] = 0.f;
             acc1[i] = 0.f;
         }
-        if (MODE == 0 && small_tile(seg, w)) {
+        if (SMALL && MODE != 2 && small_tile(seg, w)) {
             // M = 64 tile: rows 16q + j/4 ... live in lanes 0-15 of quarter q.
             // This thread holds rows rA = 16q + lane/4 and rB = rA + 8, 16
-            // gate and 16 up columns of each (its half's 64 columns, 2 per
-            // 8-column group): acc0[4i + e] / acc1[4i + e], e < 2 row rA,
-            // e >= 2 row rB, columns half*64 + 8i + 2(lane%4) + (e&1).
+            // columns of each 128-column half (its 64 columns, 2 per 8-column
+            // group): acc0[4i + e] / acc1[4i + e], e < 2 row rA, e >= 2 row
+            // rB, columns half*64 + 8i + 2(lane%4) + (e&1) of each half.
             const int gA = seg[w.e] + w.mt * BM + 16 * q + (lane >> 2), gB = gA + 8;
             const float* saA = p.a_scales + static_cast<int64_t>(gA < p.P ? gA : p.P - 1) * p.num_kb;
             const float* saB = p.a_scales + static_cast<int64_t>(gB < p.P ? gB : p.P - 1) * p.num_kb;
-            const float* s0 = p.b_s0 + (static_cast<int64_t>(w.e) * p.b_nblocks + w.nt) * p.num_kb;
-            const float* s1 = p.b_s1 + (static_cast<int64_t>(w.e) * p.b_nblocks + w.nt) * p.num_kb;
-            float aA_n = __ldg(saA), aB_n = __ldg(saB), w0_n = __ldg(s0), w1_n = __ldg(s1);
+            const int sb0 = MODE == 0 ? w.nt : 2 * w.nt;
+            const int sb1 = MODE == 0 ? w.nt : 2 * w.nt + 1;
+            const bool two = sb1 < p.b_nblocks;
+            const float* s0 = p.b_s0 + (static_cast<int64_t>(w.e) * p.b_nblocks + sb0) * p.num_kb;
+            const float* s1 = p.b_s1 + (static_cast<int64_t>(w.e) * p.b_nblocks + (two ? sb1 : sb0)) * p.num_kb;
+            float aA_n = __ldg(saA), aB_n = __ldg(saB), w0_n = __ldg(s0), w1_n = two ? __ldg(s1) : 0.f;
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
                 const float c0A = aA_n * w0_n, c0B = aB_n * w0_n;
                 const float c1A = aA_n * w1_n, c1B = aB_n * w1_n;
@@ -454,7 +520,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
                     aA_n = __ldg(saA + kb + 1);
                     aB_n = __ldg(saB + kb + 1);
                     w0_n = __ldg(s0 + kb + 1);
-                    w1_n = __ldg(s1 + kb + 1);
+                    if (two) w1_n = __ldg(s1 + kb + 1);
                 }
                 const int b = it & 1;
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tfull0 + 8 * b, (it >> 1) & 1, abort, WAIT_NS)))
@@ -472,7 +538,11 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
 #pragma unroll
                 for (int i = 0; i < 32; ++i) acc1[i] = fmaf((i & 2) ? c1B : c1A, __uint_as_float(rb[i]), acc1[i]);
             }
-            small_tail(p, w, q, half, lane, gA, gB, seg[w.e + 1], acc0, acc1, amax_x, nitem, xbar0, abort);
+            if (MODE == 0)
+                small_tail(p, w, q, half, lane, gA, gB, seg[w.e + 1], acc0, acc1, amax_x, nitem, xbar0, abort);
+            else
+                small_down_tail(p, w, half, lane, gA, gB, seg[w.e + 1], acc0, acc1,
+                                bars - OFF_BARS + OFF_STAGE + (warp - 4) * 32 * STAGE_SLOT);
             continue;
         }
         // scales of K block kb+1 are fetched while block kb is promoted
@@ -685,7 +755,7 @@ __device__ __forceinline__ void epilogue_role(const GemmParams& p, const int* se
     }
 }
 
-template <int MODE>
+template <int MODE, bool SMALL>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const GemmParams p)
@@ -761,12 +831,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if ((threadIdx.x & 31) == 0) {
             if (warp == 0) producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total_items, sbase, bars, abort);
             else if (warp == 1 || warp == 2)
-                mma_role<MODE>(p, seg, ipre, total_items, sbase, bars, tmem, abort, warp - 1);
+                mma_role<MODE, SMALL>(p, seg, ipre, total_items, sbase, bars, tmem, abort, warp - 1);
             else if (warp == 3) producer_a<MODE>(&tmA, p, seg, ipre, total_items, sbase, bars, abort);
         }
     } else {
         setmaxnreg_inc<REGS_EPI>();
-        epilogue_role<MODE>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
+        epilogue_role<MODE, SMALL>(p, seg, ipre, total_items, bars, tmem, amax_x, abort);
         // the y bulk copies must be done with shared memory (and complete)
         // before the CTA exits
         if (MODE != 0) bulk_wait_all();
@@ -886,26 +956,32 @@ bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool SMALL>
 cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                      int grid, cudaStream_t s)
 {
     const int smem = smem_bytes_for(MAX_E);
     // per device, once; host threads may launch concurrently
-    static std::atomic<bool> attr_done[64];
+    static std::atomic<bool> attr_done[64];  // one set per instantiation
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
-        err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, SMALL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
         if (dev < 64) attr_done[dev].store(true, std::memory_order_release);
     }
-    grouped_gemm_kernel<MODE><<<grid, THREADS, smem_bytes_for(p.E), s>>>(a, b0, b1, p);
+    grouped_gemm_kernel<MODE, SMALL><<<grid, THREADS, smem_bytes_for(p.E), s>>>(a, b0, b1, p);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+bool make_tmap_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  uint32_t box_rows)
+{
+    return make_tmap(m, base, rank, dims, strides_bytes, box_rows);
+}
 
 size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
                             size_t* off_sh, size_t* off_cnt, size_t* off_nv)
@@ -1006,8 +1082,13 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
     g.H = H;
     g.status = a.status;
     if ((err = stage_mark(a, 1, s)) != cudaSuccess) return err;
+    // The M = 64 variant of the gate/up and down kernels pays off when many
+    // experts receive few rows (a skewed routing of a short batch); with 256
+    // or more rows per expert on average nearly every tile is full, and the
+    // variant without that path is faster.  Both give identical bits.
+    const bool small = P < static_cast<int64_t>(E) * 256;
     if (!a.down_only) {
-        err = run_gemm<0>(tmA1, tmG, tmU, g, grid, s);
+        err = small ? run_gemm<0, true>(tmA1, tmG, tmU, g, grid, s) : run_gemm<0, false>(tmA1, tmG, tmU, g, grid, s);
         if (err != cudaSuccess) return err;
     }
 
@@ -1036,8 +1117,9 @@ cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s)
         d.k = a.k;
     }
     if ((err = stage_mark(a, 2, s)) != cudaSuccess) return err;
-    if ((err = a.fuse ? run_gemm<2>(tmA2, tmD, tmD, d, grid, s) : run_gemm<1>(tmA2, tmD, tmD, d, grid, s)) !=
-        cudaSuccess)
+    if ((err = a.fuse    ? run_gemm<2, false>(tmA2, tmD, tmD, d, grid, s)
+               : small ? run_gemm<1, true>(tmA2, tmD, tmD, d, grid, s)
+                       : run_gemm<1, false>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess)
         return err;
     return stage_mark(a, 3, s);
 }
