@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.argtypes = [P, i64, i32, i32, P, P, P, P, P]
         L.moe_route_noalloc_error.restype = ctypes.c_char_p
         L.moe_route_noalloc_error.argtypes = []
+        L.moe_quant_act_mx.restype = i32
+        L.moe_quant_act_mx.argtypes = [P, i64, i32, P, P, P]
         L.moe_quant_act.restype = i32
         L.moe_quant_act.argtypes = [P, i64, i32, P, P, P]
         L.moe_layer_workspace_bytes.restype = sz
@@ -115,6 +117,16 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_intermediate.restype = i32
         L.moe_ffn_intermediate.argtypes = [P, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p),
                                            ctypes.POINTER(ctypes.c_void_p)]
+        L.moe_ffn_mx_workspace_bytes.restype = sz
+        L.moe_ffn_mx_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+        L.moe_grouped_ffn_mx.restype = i32
+        L.moe_grouped_ffn_mx.argtypes = [P, P, i64, i32, P, P, i32, P, P, i32, i32,
+                                         P, P, P, P, P, P, P, P, sz, P, P]
+        L.moe_ffn_mx_intermediate.restype = i32
+        L.moe_ffn_mx_intermediate.argtypes = [P, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p),
+                                              ctypes.POINTER(ctypes.c_void_p)]
+        L.moe_debug_grouped_down_mx.restype = i32
+        L.moe_debug_grouped_down_mx.argtypes = [P, P, i64, i32, i32, P, P, P, i32, i32, P, P, P, P, sz, P]
         _lib = L
     return _lib
 
@@ -177,6 +189,12 @@ def moe_quant_act(x, codes, scales, stream=None):
     _check(lib().moe_quant_act(_p(x), T, H, _p(codes), _p(scales), _s(stream)), "moe_quant_act")
 
 
+def moe_quant_act_mx(x, codes, scales, stream=None):
+    """BF16 [T,H] -> MXFP8 codes uint8 [T,H] and UE8M0 scale bytes [T,H/32]."""
+    T, H = x.shape
+    _check(lib().moe_quant_act_mx(_p(x), T, H, _p(codes), _p(scales), _s(stream)), "moe_quant_act_mx")
+
+
 def moe_route_quant(logits, x, top_k, topk_ids, topk_w, expert_offsets, sorted_pairs, codes, scales, ws,
                     stream=None):
     """moe_route and moe_quant_act in one call (the quantiser rides in the
@@ -203,6 +221,51 @@ def moe_grouped_ffn(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_
                                  _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate),
                                  _p(w_up), _p(s_up), _p(w_down), _p(s_down), _p(y), _p(ws),
                                  ws.numel() * ws.element_size(), _s(stream), ev), "moe_grouped_ffn")
+
+
+def moe_ffn_mx_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> int:
+    return int(lib().moe_ffn_mx_workspace_bytes(T, H, I, E, top_k))
+
+
+def moe_grouped_ffn_mx(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs,
+                       w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None, stage_events=None):
+    """The MXFP8 experts: uint8 codes with uint8 UE8M0 scale bytes per 32
+    values (act_scales [T, H/32], s_gate/s_up [E, I, H/32], s_down [E, H, I/32])."""
+    T, H = codes.shape
+    E, I, _ = w_gate.shape
+    top_k = topk_ids.shape[1]
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * 4)(*[e.cuda_event for e in stage_events])
+    _check(lib().moe_grouped_ffn_mx(_p(codes), _p(act_scales), T, H, _p(topk_ids), _p(topk_w), top_k,
+                                    _p(expert_offsets), _p(sorted_pairs), E, I, _p(w_gate), _p(s_gate),
+                                    _p(w_up), _p(s_up), _p(w_down), _p(s_down), _p(y), _p(ws),
+                                    ws.numel() * ws.element_size(), _s(stream), ev), "moe_grouped_ffn_mx")
+
+
+def moe_ffn_mx_intermediate(ws, T: int, H: int, I: int, top_k: int):
+    """(codes [T*top_k, Ip] uint8, scale bytes [T*top_k, Ip/32] uint8) views
+    of the MX intermediate held in an MX FFN workspace, rows in expert order."""
+    c, sc = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib().moe_ffn_mx_intermediate(_p(ws), T, H, I, top_k, ctypes.byref(c), ctypes.byref(sc)),
+           "moe_ffn_mx_intermediate")
+    Ip = (I + 127) // 128 * 128
+    base = ws.data_ptr()
+    oc, osc = c.value - base, sc.value - base
+    P = T * top_k
+    return ws[oc: oc + P * Ip].view(P, Ip), ws[osc: osc + P * (Ip // 32)].view(P, Ip // 32)
+
+
+def moe_debug_grouped_down_mx(h_codes, h_scales, topk_w, expert_offsets, sorted_pairs, w_down, s_down, y, ws,
+                              stream=None):
+    """Test hook: the MX down GEMM alone on a caller-supplied intermediate
+    (h_codes [T*top_k, Ip] uint8, h_scales [T*top_k, Ip/32] uint8, expert
+    order), writing y [T, top_k, H] for the valid pairs."""
+    T, k = topk_w.shape
+    E, H, I = w_down.shape
+    _check(lib().moe_debug_grouped_down_mx(_p(h_codes), _p(h_scales), T, H, k, _p(topk_w), _p(expert_offsets),
+                                           _p(sorted_pairs), E, I, _p(w_down), _p(s_down), _p(y), _p(ws),
+                                           ws.numel(), _s(stream)), "moe_debug_grouped_down_mx")
 
 
 def moe_combine(y, topk_ids, num_experts, routed_scaling, out_f32, out_bf16, ws, stream=None):

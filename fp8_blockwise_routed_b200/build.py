@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfp8moe.so")
-SOURCES = ["api.cu", "route.cu", "quant_act.cu", "combine.cu", "grouped_ffn.cu", "layer.cu", "ep.cu"]
-HEADERS = ["internal.h", "sm100.cuh", "quant_body.cuh"]
+SOURCES = ["api.cu", "route.cu", "quant_act.cu", "combine.cu", "grouped_ffn.cu", "layer.cu", "ep.cu", "grouped_mx.cu"]
+HEADERS = ["internal.h", "sm100.cuh", "quant_body.cuh", "mx_rule.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

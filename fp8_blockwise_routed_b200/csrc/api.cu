@@ -89,6 +89,18 @@ size_t route_layout(int64_t T, int E, int k, size_t* off_arr, size_t* off_hist, 
     return route_ws_layout(T, E, k, off_arr, off_hist, off_rank);
 }
 
+// Shape and pointer checks shared by the MX FFN entry points.
+int mx_check(int64_t T, int H, int I, int E, int top_k, const void* ws)
+{
+    if (T < 0 || H < 128 || H > MOE_MAX_HIDDEN || H % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOP_K) return MOE_ERR_INVALID_ARG;
+    if (I < 128 || I > MOE_MAX_INTERMEDIATE) return MOE_ERR_INVALID_ARG;
+    if (I % 32 != 0) return MOE_ERR_UNSUPPORTED;  // one scale byte per 32 intermediate columns
+    if (T * top_k > (int64_t(1) << 31) - 1) return MOE_ERR_UNSUPPORTED;
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -183,6 +195,17 @@ int moe_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* sc
     if (int r = check_device()) return r;
     cudaError_t err = launch_quant_act(x, T, H, codes, scales, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quant_act");
+}
+
+int moe_quant_act_mx(const uint16_t* x, int64_t T, int H, uint8_t* codes, uint8_t* scales, void* stream)
+{
+    if (T < 0 || H < 32 || H > MOE_MAX_HIDDEN || H % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !codes || !scales)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return MOE_ERR_ALIGNMENT;
+    if (T == 0) return MOE_OK;
+    if (int r = check_device()) return r;
+    cudaError_t err = launch_quant_mx(x, T, H, codes, scales, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quant_act_mx");
 }
 
 size_t moe_ffn_workspace_bytes(int64_t T, int H, int I, int E, int top_k)
@@ -421,6 +444,113 @@ int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales, int64_
     a.down_only = 1;
     cudaError_t err = launch_grouped_ffn(a, s);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_grouped_down");
+}
+
+
+size_t moe_ffn_mx_workspace_bytes(int64_t T, int H, int I, int E, int top_k)
+{
+    (void)E;
+    if (T < 0 || H < 128 || I < 1 || top_k < 0) return 0;
+    size_t a, b, c, d;
+    return ffn_mx_workspace_layout(T, H, I, top_k, &a, &b, &c, &d);
+}
+
+int moe_grouped_ffn_mx(const uint8_t* codes, const uint8_t* act_scales, int64_t T, int H, const int32_t* topk_ids,
+                       const float* topk_w, int top_k, const int32_t* expert_offsets, const int32_t* sorted_pairs,
+                       int E, int I, const uint8_t* w_gate, const uint8_t* s_gate, const uint8_t* w_up,
+                       const uint8_t* s_up, const uint8_t* w_down, const uint8_t* s_down, float* y, void* ws,
+                       size_t ws_bytes, void* stream, void* const* stage_events)
+{
+    if (int r = mx_check(T, H, I, E, top_k, ws)) return r;
+    if (T > 0 && (!codes || !act_scales || !topk_ids || !topk_w || !expert_offsets || !sorted_pairs || !w_gate ||
+                  !s_gate || !w_up || !s_up || !w_down || !s_down || !y))
+        return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs, w_gate, s_gate,
+                          w_up, s_up, w_down, s_down, y, ws};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
+    size_t off_a, off_sa, off_h, off_sh;
+    if (ws_bytes < ffn_mx_workspace_layout(T, H, I, top_k, &off_a, &off_sa, &off_h, &off_sh))
+        return MOE_ERR_WORKSPACE;
+    if (int r = check_device()) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int r = clear_status(ws, s)) return r;
+    if (T == 0) return MOE_OK;
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    FfnMxArgs a{};
+    a.codes = codes;
+    a.act_scales = act_scales;
+    a.T = T;
+    a.H = H;
+    a.topk_ids = topk_ids;
+    a.topk_w = topk_w;
+    a.k = top_k;
+    a.expert_offsets = expert_offsets;
+    a.sorted_pairs = sorted_pairs;
+    a.E = E;
+    a.I = I;
+    a.w_gate = w_gate;
+    a.s_gate = s_gate;
+    a.w_up = w_up;
+    a.s_up = s_up;
+    a.w_down = w_down;
+    a.s_down = s_down;
+    a.y = y;
+    a.status = reinterpret_cast<int*>(w8);
+    a.a_sorted = w8 + off_a;
+    a.sa_sorted = w8 + off_sa;
+    a.h_codes = w8 + off_h;
+    a.h_scales = w8 + off_sh;
+    a.stage_events = stage_events;
+    cudaError_t err = launch_grouped_ffn_mx(a, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_ffn_mx");
+}
+
+int moe_ffn_mx_intermediate(const void* ws, int64_t T, int H, int I, int top_k, const uint8_t** h_codes,
+                            const uint8_t** h_scales)
+{
+    if (!ws || !h_codes || !h_scales || T < 0 || H < 128 || I < 1 || top_k < 1) return MOE_ERR_INVALID_ARG;
+    size_t off_a, off_sa, off_h, off_sh;
+    ffn_mx_workspace_layout(T, H, I, top_k, &off_a, &off_sa, &off_h, &off_sh);
+    *h_codes = static_cast<const uint8_t*>(ws) + off_h;
+    *h_scales = static_cast<const uint8_t*>(ws) + off_sh;
+    return MOE_OK;
+}
+
+int moe_debug_grouped_down_mx(const uint8_t* h_codes, const uint8_t* h_scales, int64_t T, int H, int top_k,
+                              const float* topk_w, const int32_t* expert_offsets, const int32_t* sorted_pairs, int E,
+                              int I, const uint8_t* w_down, const uint8_t* s_down, float* y, void* ws,
+                              size_t ws_bytes, void* stream)
+{
+    if (int r = mx_check(T, H, I, E, top_k, ws)) return r;
+    if (T > 0 && (!h_codes || !h_scales || !topk_w || !expert_offsets || !sorted_pairs || !w_down || !s_down || !y))
+        return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {h_codes, h_scales, topk_w, expert_offsets, sorted_pairs, w_down, s_down, y, ws};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    if (int r = check_device()) return r;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int r = clear_status(ws, s)) return r;
+    if (T == 0) return MOE_OK;
+    FfnMxArgs a{};
+    a.T = T;
+    a.H = H;
+    a.topk_w = topk_w;
+    a.k = top_k;
+    a.expert_offsets = expert_offsets;
+    a.sorted_pairs = sorted_pairs;
+    a.E = E;
+    a.I = I;
+    a.w_down = w_down;
+    a.s_down = s_down;
+    a.y = y;
+    a.status = static_cast<int*>(ws);
+    a.h_codes = const_cast<uint8_t*>(h_codes);
+    a.h_scales = const_cast<uint8_t*>(h_scales);
+    a.down_only = 1;
+    cudaError_t err = launch_grouped_ffn_mx(a, s);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_debug_grouped_down_mx");
 }
 
 int moe_ffn_intermediate(const void* ws, int64_t T, int H, int I, int top_k, const uint8_t** h_codes,

@@ -1,9 +1,11 @@
 // internal.h -- launchers shared between the kernel files and the C ABI.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (types only; libcuda is not linked)
+#include <cuda_runtime.h>
+
 #include <cstddef>
 #include <cstdint>
-#include <cuda_runtime.h>
 
 namespace fp8moe {
 
@@ -60,6 +62,8 @@ bool device_info(DeviceInfo* out);
 
 cudaError_t launch_quant_act(const uint16_t* x, int64_t T, int H, uint8_t* codes, float* scales, cudaStream_t s);
 cudaError_t launch_encode(const float* in, int64_t n, uint8_t* out, cudaStream_t s);
+// MXFP8 activations: codes [T, H] and one UE8M0 scale byte per 32 values [T, H/32].
+cudaError_t launch_quant_mx(const uint16_t* x, int64_t T, int H, uint8_t* codes, uint8_t* scales, cudaStream_t s);
 
 // Activation quantiser work carried by the route's top-k launch.
 struct QuantArgs {
@@ -136,5 +140,44 @@ size_t ffn_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_
 // Returns cudaSuccess, or an error (including cudaErrorNotSupported when the
 // tensor-map encoder cannot be obtained).
 cudaError_t launch_grouped_ffn(const FfnArgs& a, cudaStream_t s);
+
+// Row-major uint8 tensor map of `rank` (2 or 3) dims, innermost first, tile
+// box 128 bytes x box_rows (x 1), 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  uint32_t box_rows);
+
+// MXFP8 expert FFN (moe_grouped_ffn_mx): MX codes and UE8M0 scale bytes for
+// activations [T, H/32], gate/up weights [E, I, H/32] and down weights
+// [E, H, I/32]; the same routing inputs and y output as FfnArgs.
+struct FfnMxArgs {
+    const uint8_t* codes;
+    const uint8_t* act_scales;  // [T, H/32]
+    int64_t T;
+    int H;
+    const int32_t* topk_ids;
+    const float* topk_w;
+    int k;
+    const int32_t* expert_offsets;
+    const int32_t* sorted_pairs;
+    int E;
+    int I;
+    const uint8_t* w_gate;
+    const uint8_t* s_gate;  // [E, I, H/32]
+    const uint8_t* w_up;
+    const uint8_t* s_up;
+    const uint8_t* w_down;
+    const uint8_t* s_down;  // [E, H, I/32]
+    float* y;               // [T, k, H]
+    int* status;
+    uint8_t* a_sorted;      // [P, H] codes in expert order
+    uint8_t* sa_sorted;     // [P, H/32] scale bytes in expert order
+    uint8_t* h_codes;       // [P, Ip]
+    uint8_t* h_scales;      // [P, Ip/32]
+    void* const* stage_events;
+    int down_only;          // 1: h_codes / h_scales are inputs; only the down GEMM runs
+};
+size_t ffn_mx_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
+                               size_t* off_sh);
+cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s);
 
 }  // namespace fp8moe

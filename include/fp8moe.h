@@ -212,6 +212,26 @@ MOE_API int moe_quant_act(const uint16_t* x, int64_t T, int H,
                   uint8_t* codes, float* scales, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_quant_act_mx -- BF16 activations to MXFP8: E4M3 codes with one UE8M0
+ * (power-of-two) scale byte per 32 consecutive values.  The pages name an
+ * MXFP8 MoE runtime only as not yet qualified ("Exact AVX2 FP8 arithmetic
+ * conversion avoids costly LUT gathers", "Real-checkpoint measurements",
+ * caveats); the rule follows the OCP Microscaling Formats:
+ *   amax = max |x| over the block; se = floor(log2(amax)) - 8 (8: the
+ *   exponent of E4M3's largest value, 448 = 1.75 * 2^8), clamped to
+ *   [-127, 127], -127 for amax = 0; scale byte = se + 127 (value 2^se);
+ *   code = E4M3(x / 2^se), round to nearest even, saturating at +-448; a
+ *   block holding NaN or Inf gets scale byte 0xFF and every code 0x7F.
+ *
+ *   x       [T, H]     BF16 (raw 16-bit words), read
+ *   codes   [T, H]     uint8 E4M3, written
+ *   scales  [T, H/32]  uint8 UE8M0, written
+ *
+ * Limits: T >= 0, H % 32 == 0, 32 <= H <= 16384.
+ * ------------------------------------------------------------------------- */
+MOE_API int moe_quant_act_mx(const uint16_t* x, int64_t T, int H, uint8_t* codes, uint8_t* scales, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_grouped_ffn -- the experts: grouped gate/up GEMM -> SiLU*up ->
  * requantise -> grouped down GEMM -> routing-weighted slot rows.
  *
@@ -262,6 +282,46 @@ MOE_API int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64
                     const uint8_t* w_down, const float* s_down,
                     float* y, void* ws, size_t ws_bytes, void* stream,
                     void* const* stage_events);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_ffn_mx -- the experts of the MXFP8 variant: the same routing
+ * inputs, steps and y output as moe_grouped_ffn, with every operand in the
+ * OCP MX format (E4M3 codes, one UE8M0 scale byte per 32 values along K)
+ * and the scales applied by the tensor core inside each K = 32 step.  The
+ * pages list an MXFP8 MoE runtime only as not yet qualified ("Exact AVX2 FP8
+ * arithmetic conversion avoids costly LUT gathers", "Real-checkpoint
+ * measurements", caveats); the arithmetic follows the OCP Microscaling
+ * Formats.  For every valid pair (token t, slot j, expert e):
+ *   g[n] = sum_k 2^(sa[t,k/32]-127) dec(q[t,k]) 2^(sg[e,n,k/32]-127) dec(Wg[e,n,k])
+ *   u[n] likewise with Wu, su;                         (FP32 accumulation)
+ *   h[n] = g[n] / (1 + exp(-g[n])) * u[n]              (unclamped SiLU)
+ *   (hq, sh) = the moe_quant_act_mx rule applied to h per 32 columns
+ *   o[c] = sum_i 2^(sh[i/32]-127) dec(hq[i]) 2^(sd[e,c,i/32]-127) dec(Wd[e,c,i])
+ *   y[t, j, c] = topk_w[t, j] * o[c]
+ * Rows of y for slots with id -1 are not written; each row's bits depend
+ * only on that row's inputs and the expert's weights.  Follow with
+ * moe_combine.
+ *
+ *   codes, act_scales      [T, H] uint8, [T, H/32] uint8  (moe_quant_act_mx output)
+ *   topk_ids, topk_w, expert_offsets, sorted_pairs   as moe_grouped_ffn
+ *   w_gate, w_up           [E, I, H] uint8 E4M3;  s_gate, s_up [E, I, H/32] uint8 UE8M0
+ *   w_down                 [E, H, I] uint8 E4M3;  s_down       [E, H, I/32] uint8 UE8M0
+ *   y                      [T, top_k, H] FP32, written (valid slots only)
+ *   ws, ws_bytes           scratch of at least moe_ffn_mx_workspace_bytes(T, H, I, E, top_k)
+ *   stage_events           as moe_grouped_ffn
+ *
+ * Limits: H % 128 == 0, 128 <= H <= 16384; I % 32 == 0, 128 <= I <= 8192;
+ * 1 <= E <= 1024; 1 <= top_k <= min(E, 32); T >= 0.  Scale bytes 0xFF (NaN)
+ * and code bytes 0x7F/0xFF in the weights are outside the contract.
+ * Errors as moe_grouped_ffn.
+ * ------------------------------------------------------------------------- */
+MOE_API size_t moe_ffn_mx_workspace_bytes(int64_t T, int H, int I, int E, int top_k);
+MOE_API int moe_grouped_ffn_mx(const uint8_t* codes, const uint8_t* act_scales, int64_t T, int H,
+                               const int32_t* topk_ids, const float* topk_w, int top_k,
+                               const int32_t* expert_offsets, const int32_t* sorted_pairs, int E, int I,
+                               const uint8_t* w_gate, const uint8_t* s_gate, const uint8_t* w_up,
+                               const uint8_t* s_up, const uint8_t* w_down, const uint8_t* s_down, float* y,
+                               void* ws, size_t ws_bytes, void* stream, void* const* stage_events);
 
 /* ---------------------------------------------------------------------------
  * moe_combine -- out[t, :] = routed_scaling * sum_{j : id(t,j) >= 0} y[t, j, :]
@@ -488,6 +548,25 @@ MOE_API int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales
                                    const float* topk_w, const int32_t* expert_offsets, const int32_t* sorted_pairs,
                                    int E, int I, const uint8_t* w_down, const float* s_down, float* y, void* ws,
                                    size_t ws_bytes, void* stream);
+
+/* moe_ffn_mx_intermediate: device pointers into a workspace last used by
+ * moe_grouped_ffn_mx with the same (T, H, I, top_k): the MX intermediate
+ * codes [T*top_k, Ip] (columns I..Ip-1 unspecified, Ip = ceil(I/128)*128)
+ * and scale bytes [T*top_k, Ip/32] (bytes I/32.. unspecified), rows in
+ * expert order.  Host arithmetic only. */
+MOE_API int moe_ffn_mx_intermediate(const void* ws, int64_t T, int H, int I, int top_k,
+                                    const uint8_t** h_codes, const uint8_t** h_scales);
+
+/* moe_debug_grouped_down_mx: the down GEMM of moe_grouped_ffn_mx alone, on
+ * an intermediate the caller supplies in the layout moe_ffn_mx_intermediate
+ * describes (h_codes [T*top_k, Ip], h_scales [T*top_k, Ip/32], expert
+ * order).  Writes y as moe_grouped_ffn_mx's down stage does (same kernel).
+ * Workspace: at least moe_combine_workspace_bytes().  Limits and errors as
+ * moe_grouped_ffn_mx. */
+MOE_API int moe_debug_grouped_down_mx(const uint8_t* h_codes, const uint8_t* h_scales, int64_t T, int H,
+                                      int top_k, const float* topk_w, const int32_t* expert_offsets,
+                                      const int32_t* sorted_pairs, int E, int I, const uint8_t* w_down,
+                                      const uint8_t* s_down, float* y, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }
