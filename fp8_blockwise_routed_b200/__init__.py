@@ -117,6 +117,10 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_intermediate.restype = i32
         L.moe_ffn_intermediate.argtypes = [P, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p),
                                            ctypes.POINTER(ctypes.c_void_p)]
+        L.moe_mx_packed_scales_bytes.restype = sz
+        L.moe_mx_packed_scales_bytes.argtypes = [i64, i32, i32]
+        L.moe_mx_pack_scales.restype = i32
+        L.moe_mx_pack_scales.argtypes = [P, i64, i32, i32, P, P]
         L.moe_ffn_mx_workspace_bytes.restype = sz
         L.moe_ffn_mx_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
         L.moe_grouped_ffn_mx.restype = i32
@@ -223,6 +227,18 @@ def moe_grouped_ffn(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_
                                  ws.numel() * ws.element_size(), _s(stream), ev), "moe_grouped_ffn")
 
 
+def moe_mx_pack_scales(src, stream=None):
+    """MX weight scales [E, R, K/32] uint8 (CUDA) -> the packed layout the MX
+    FFN reads: a new uint8 tensor [E, ceil(K/512), R, 16]."""
+    E, R, C = src.shape
+    K = C * 32
+    G = (K + 511) // 512
+    assert int(lib().moe_mx_packed_scales_bytes(E, R, K)) == E * G * R * 16
+    dst = torch.empty((E, G, R, 16), dtype=torch.uint8, device=src.device)
+    _check(lib().moe_mx_pack_scales(_p(src.contiguous()), E, R, K, _p(dst), _s(stream)), "moe_mx_pack_scales")
+    return dst
+
+
 def moe_ffn_mx_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> int:
     return int(lib().moe_ffn_mx_workspace_bytes(T, H, I, E, top_k))
 
@@ -230,7 +246,8 @@ def moe_ffn_mx_workspace_bytes(T: int, H: int, I: int, E: int, top_k: int) -> in
 def moe_grouped_ffn_mx(codes, act_scales, topk_ids, topk_w, expert_offsets, sorted_pairs,
                        w_gate, s_gate, w_up, s_up, w_down, s_down, y, ws, stream=None, stage_events=None):
     """The MXFP8 experts: uint8 codes with uint8 UE8M0 scale bytes per 32
-    values (act_scales [T, H/32], s_gate/s_up [E, I, H/32], s_down [E, H, I/32])."""
+    values (act_scales [T, H/32]; s_gate, s_up, s_down as moe_mx_pack_scales
+    returns them)."""
     T, H = codes.shape
     E, I, _ = w_gate.shape
     top_k = topk_ids.shape[1]
@@ -244,8 +261,9 @@ def moe_grouped_ffn_mx(codes, act_scales, topk_ids, topk_w, expert_offsets, sort
 
 
 def moe_ffn_mx_intermediate(ws, T: int, H: int, I: int, top_k: int):
-    """(codes [T*top_k, Ip] uint8, scale bytes [T*top_k, Ip/32] uint8) views
-    of the MX intermediate held in an MX FFN workspace, rows in expert order."""
+    """(codes [T*top_k, Ip] uint8, scale bytes [G, T*top_k, 16] uint8 with
+    G = ceil(Ip/512): chunk c of row r at [c // 16, r, c % 16]) views of the
+    MX intermediate held in an MX FFN workspace, rows in expert order."""
     c, sc = ctypes.c_void_p(), ctypes.c_void_p()
     _check(lib().moe_ffn_mx_intermediate(_p(ws), T, H, I, top_k, ctypes.byref(c), ctypes.byref(sc)),
            "moe_ffn_mx_intermediate")
@@ -253,14 +271,16 @@ def moe_ffn_mx_intermediate(ws, T: int, H: int, I: int, top_k: int):
     base = ws.data_ptr()
     oc, osc = c.value - base, sc.value - base
     P = T * top_k
-    return ws[oc: oc + P * Ip].view(P, Ip), ws[osc: osc + P * (Ip // 32)].view(P, Ip // 32)
+    G = (Ip + 511) // 512
+    return ws[oc: oc + P * Ip].view(P, Ip), ws[osc: osc + G * P * 16].view(G, P, 16)
 
 
 def moe_debug_grouped_down_mx(h_codes, h_scales, topk_w, expert_offsets, sorted_pairs, w_down, s_down, y, ws,
                               stream=None):
     """Test hook: the MX down GEMM alone on a caller-supplied intermediate
-    (h_codes [T*top_k, Ip] uint8, h_scales [T*top_k, Ip/32] uint8, expert
-    order), writing y [T, top_k, H] for the valid pairs."""
+    (h_codes [T*top_k, Ip] uint8, h_scales [G, T*top_k, 16] uint8 as
+    moe_ffn_mx_intermediate lays it out, expert order), writing y
+    [T, top_k, H] for the valid pairs."""
     T, k = topk_w.shape
     E, H, I = w_down.shape
     _check(lib().moe_debug_grouped_down_mx(_p(h_codes), _p(h_scales), T, H, k, _p(topk_w), _p(expert_offsets),

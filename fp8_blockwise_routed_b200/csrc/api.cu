@@ -447,6 +447,23 @@ int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales, int64_
 }
 
 
+size_t moe_mx_packed_scales_bytes(int64_t E, int R, int K)
+{
+    if (E < 0 || R < 1 || K < 32 || K % 32 != 0) return 0;
+    return static_cast<size_t>(E) * mx_scale_groups(K) * R * 16;
+}
+
+int moe_mx_pack_scales(const uint8_t* src, int64_t E, int R, int K, uint8_t* dst, void* stream)
+{
+    if (E < 0 || R < 1 || K < 32 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (E > 0 && (!src || !dst)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(dst)) return MOE_ERR_ALIGNMENT;
+    if (E == 0) return MOE_OK;
+    if (int r = check_device()) return r;
+    cudaError_t err = launch_pack_mx_scales(src, E, R, K, dst, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_mx_pack_scales");
+}
+
 size_t moe_ffn_mx_workspace_bytes(int64_t T, int H, int I, int E, int top_k)
 {
     (void)E;

@@ -12,9 +12,13 @@
 //
 // Launch sequence of one moe_grouped_ffn_mx call (stream-ordered):
 //   gather   : A code rows and their scale bytes in expert order
-//   gate/up  : tile 128 rows x (64 gate + 64 up) columns; epilogue
+//   gate/up  : tile 128 rows x (96 gate + 96 up) columns; epilogue
 //              h = SiLU(g) * u, MX-requantised per 32 columns
-//   down     : tile 128 rows x 128 output columns; epilogue y[pair] = w * o
+//   down     : tile 128 rows x 192 output columns; epilogue y[pair] = w * o
+// N = 192 is the widest tile for which two accumulators and the scale ring
+// fit the 512 TMEM columns; it reads 40 KB of operands per 128-deep K block
+// for 6.3 MFLOP, so the tensor pipe, not the shared-memory fill, sets the
+// pace of a K block.
 //
 // Warp roles (384 threads, one CTA per SM, persistent over work items ordered
 // expert-major, then n-tile, then m-tile):
@@ -22,16 +26,21 @@
 //   warp 1      MMA issuer (one lane; also allocates TMEM)
 //   warp 3      activation TMA producer (one lane)
 //   warps 4..7  epilogue: warp w drains TMEM lanes 32*(w%4), once per item
-//   warps 8..11 scale stagers: per K block, write the tile's A and B scale
-//               bytes into a TMEM ring with tcgen05.st.  The MMA reads a
-//               row's scale from the lane of that row in every 32-lane
-//               sub-partition, so each of the four warps writes the same
-//               data into its own sub-partition.
-// TMEM: two 128-column accumulators (items alternate) and SF_SLOTS slots of
-// 8 scale columns.  Scale layout (K block of 128 = 4 chunks of 32): row m of
-// the A tile -> lanes m%32 (+32 per sub-partition), column m/32, byte j =
-// chunk j; B row n likewise in the slot's columns 4..7.  The MMA of chunk j
-// selects byte j (scale-factor id j).
+//   warp 2      scale loader (all lanes): the tile's A and B scale bytes of
+//               each K block from global memory into a shared ring, four K
+//               blocks per 16-byte load, the next group's loads in flight
+//   warps 8..11 scale writers: per K block, copy the shared slot into a
+//               TMEM ring with tcgen05.st.  The MMA reads a row's scale from
+//               the lane of that row in every 32-lane sub-partition, so each
+//               of the four warps writes the same data into its own
+//               sub-partition.  A tcgen05 wait also waits for the warp's
+//               outstanding global loads, hence the split: the writers keep
+//               none in flight.
+// TMEM: two 192-column accumulators (items alternate) and SF_SLOTS slots of
+// 16 scale columns.  Scale layout (K block of 128 = 4 chunks of 32): row m of
+// the A tile -> lanes m%32 (+32 per sub-partition), slot column m/32, byte
+// j = chunk j; B row n likewise in the slot's columns 8 + n/32.  The MMA of
+// chunk j selects byte j (scale-factor id j).
 // Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
 // MOE_DEV_WAIT_TIMEOUT and frees TMEM.
 #include <cuda.h>
@@ -49,15 +58,18 @@ namespace {
 using namespace sm100;
 
 constexpr int MX_BM = 128;
+constexpr int MX_BN = 192;            // MMA N: output columns of a tile
+constexpr int MX_HALF = MX_BN / 2;    // gate/up: 96 gate + 96 up weight rows
 constexpr int MX_BK = 128;
-constexpr int MX_STAGES = 6;
-constexpr int MX_A_TILE = 128 * 128;  // 16 KiB
-constexpr int MX_B_TILE = 128 * 128;  // 16 KiB
+constexpr int MX_STAGES = 5;
+constexpr int MX_A_TILE = MX_BM * MX_BK;  // 16 KiB
+constexpr int MX_B_TILE = MX_BN * MX_BK;  // 24 KiB
 constexpr int MX_STAGE = MX_A_TILE + MX_B_TILE;
 constexpr int MX_THREADS = 384;
-constexpr int SF_SLOTS = 16;
-constexpr int SF_COL = 256;             // scale ring starts after the two accumulators
-constexpr uint32_t MX_TMEM_COLS = 512;  // 2 x 128 + 16 x 8 = 384 used
+constexpr int SF_SLOTS = 8;
+constexpr int SF_SLOT_COLS = 16;              // A: columns 0..3, B: columns 8..13
+constexpr int SF_COL = 2 * MX_BN;             // the scale ring follows the two accumulators
+constexpr uint32_t MX_TMEM_COLS = 512;
 constexpr uint64_t MX_WAIT_NS = 2000000000ull;
 constexpr int MX_MAX_E = 1024;
 
@@ -65,32 +77,38 @@ constexpr int MB_FULL = 0;                       // [stages]: both producers (ar
 constexpr int MB_EMPTY = MB_FULL + MX_STAGES;    // [stages]: MMA commit
 constexpr int MB_SFF = MB_EMPTY + MX_STAGES;     // [slots]: the four stager warps
 constexpr int MB_SFE = MB_SFF + SF_SLOTS;        // [slots]: MMA commit
-constexpr int MB_AF = MB_SFE + SF_SLOTS;         // [2]: accumulator full (MMA commit)
+constexpr int MB_SSF = MB_SFE + SF_SLOTS;        // [slots]: scale loader filled the shared slot
+constexpr int MB_SSE = MB_SSF + SF_SLOTS;        // [slots]: the four writers read it
+constexpr int MB_AF = MB_SSE + SF_SLOTS;         // [2]: accumulator full (MMA commit)
 constexpr int MB_AE = MB_AF + 2;                 // [2]: accumulator drained (four epilogue warps)
 constexpr int MB_N = MB_AE + 2;
-constexpr int MX_OFF_BARS = MX_STAGES * MX_STAGE;
+constexpr int SF_WORDS = 10;                   // per lane and K block: 4 A + 6 B scale words
+constexpr int MX_OFF_SFS = MX_STAGES * MX_STAGE;  // shared scale ring [slot][word][lane]
+constexpr int MX_OFF_BARS = MX_OFF_SFS + SF_SLOTS * SF_WORDS * 32 * 4;
 constexpr int MX_OFF_MISC = MX_OFF_BARS + MB_N * 8;
 constexpr int MX_OFF_SEG = MX_OFF_MISC + 16;  // [E+1] offsets, then [E+1] item prefix
 constexpr int mx_smem_bytes(int E) { return MX_OFF_SEG + 2 * (E + 1) * 4 + 1024; }
-static_assert(SF_COL + SF_SLOTS * 8 <= static_cast<int>(MX_TMEM_COLS), "scale ring exceeds TMEM");
+static_assert(SF_COL + SF_SLOTS * SF_SLOT_COLS <= static_cast<int>(MX_TMEM_COLS), "scale ring exceeds TMEM");
+static_assert(MX_STAGE % 1024 == 0 && MX_A_TILE % 1024 == 0 && (MX_HALF * 128) % 1024 == 0,
+              "128-byte-swizzled tiles need 1024-byte alignment");
 
 struct MxParams {
     int E;
     int num_kb;            // K blocks of 128
+    int num_groups;        // groups of four K blocks: ceil(num_kb / 4)
     int n_tiles;           // output tiles per expert
     int64_t P;             // rows of the pair buffers (T * top_k)
     const int32_t* offsets;
-    const uint8_t* a_sf;   // [P, a_sf_stride] scale bytes of the A rows (expert order)
-    int a_sf_stride;       // bytes per A scale row
+    const uint8_t* a_sf;   // A rows' scale bytes (expert order), K-group-major:
+                           // [ceil(K/512)][P][16], 16 = four K blocks of four chunks
     int a_chunks;          // valid 32-column chunks of an A row (K / 32)
-    const uint8_t* b_sf0;  // gate/up: s_gate; down: s_down ([E, b_rows, b_sf_stride])
+    const uint8_t* b_sf0;  // gate/up: s_gate; down: s_down, packed [E][ceil(K/512)][b_rows][16]
     const uint8_t* b_sf1;  // gate/up: s_up
     int b_rows;            // weight rows per expert (I or H)
-    int b_sf_stride;       // bytes per weight scale row (H/32 or I/32)
     int b_chunks;          // valid chunks of a weight row (K / 32)
     // gate/up epilogue
     uint8_t* h_codes;      // [P, Ip]
-    uint8_t* h_scales;     // [P, Ip/32]
+    uint8_t* h_scales;     // [ceil(Ip/512)][P][16], the layout of a_sf
     int Ip;
     int I;
     // down epilogue
@@ -157,20 +175,6 @@ __device__ __forceinline__ void tmem_st32x8(uint32_t taddr, const uint32_t (&v)[
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Four scale bytes of one row for the K block starting at chunk c0 (of nvalid
-// chunks); missing chunks read as 127 (2^0), so zero operands stay zero.
-__device__ __forceinline__ uint32_t load_sf4(const uint8_t* row, int c0, int nvalid, bool aligned4)
-{
-    if (aligned4 && c0 + 4 <= nvalid) return __ldg(reinterpret_cast<const uint32_t*>(row + c0));
-    uint32_t v = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t b = (c0 + j < nvalid) ? static_cast<uint32_t>(__ldg(row + c0 + j)) : 127u;
-        v |= b << (8 * j);
-    }
-    return v;
-}
-
 // ---------------------------------------------------------------- roles
 
 template <int MODE>
@@ -191,11 +195,11 @@ __device__ __forceinline__ void mx_producer_b(const CUtensorMap* tm0, const CUte
             const uint32_t fb = bars + 8 * (MB_FULL + s);
             mbar_arrive_expect_tx(fb, MX_B_TILE);
             const uint32_t dst = sbase + s * MX_STAGE + MX_A_TILE;
-            if (MODE == 0) {  // 64 gate rows, then 64 up rows, of n-tile nt
-                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * 64, w.e, fb);
-                tma_load_3d(dst + MX_B_TILE / 2, tm1, kb * MX_BK, w.nt * 64, w.e, fb);
+            if (MODE == 0) {  // 96 gate rows, then 96 up rows, of n-tile nt
+                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * MX_HALF, w.e, fb);
+                tma_load_3d(dst + MX_B_TILE / 2, tm1, kb * MX_BK, w.nt * MX_HALF, w.e, fb);
             } else {
-                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * 128, w.e, fb);
+                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * MX_BN, w.e, fb);
             }
         }
     }
@@ -235,64 +239,182 @@ __device__ __forceinline__ void mx_producer_a(const CUtensorMap* tmA, const MxPa
     }
 }
 
-// Scale stager (warps 8..11, all lanes): per K block, lane t of the warp on
-// sub-partition q writes lane 32q + t of the slot: columns 0..3 the A scales
-// of tile rows t, t+32, t+64, t+96; columns 4..7 those of B rows t .. t+96.
+// Scale words for lane t: the A scales of tile rows t, t+32, t+64, t+96
+// (words 0..3) and the B scales of rows t, t+32, .., t+160 (words 4..9),
+// four K chunks (one K block) per 32-bit word.  Both operands' scales are
+// K-group-major ([groups][rows][16 bytes], a group = four K blocks), so the
+// loader fetches a group of four K blocks of 32 consecutive rows with one
+// coalesced 16-byte-per-lane load.  A cursor walks this CTA's (item, group)
+// sequence.
+struct SfGroup {
+    int item, kb0, row0;
+    MxItem w;
+};
+
+__device__ __forceinline__ void sf_group_next(SfGroup& c, const MxParams& p, const int* seg, const int* ipre,
+                                              int total)
+{
+    c.kb0 += 4;
+    if (c.kb0 < p.num_kb) return;
+    c.kb0 = 0;
+    c.item += gridDim.x;
+    if (c.item < total) {
+        c.w = mx_decode(seg, ipre, p.E, c.item);
+        c.row0 = seg[c.w.e] + c.w.mt * MX_BM;
+    }
+}
+
+// Chunks at or beyond nvalid of the 16-byte group starting at chunk c0 read
+// as 127 (2^0): K padding, whose codes are zero.
+__device__ __forceinline__ uint4 mask_sf16(uint4 v, int c0, int nvalid)
+{
+    if (c0 + 16 <= nvalid) return v;
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int b = 0; b < 16; ++b)
+        if (c0 + b >= nvalid) w[b >> 2] = (w[b >> 2] & ~(0xFFu << (8 * (b & 3)))) | (0x7Fu << (8 * (b & 3)));
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <int MODE>
-__device__ __forceinline__ void mx_stager(const MxParams& p, const int* seg, const int* ipre, int total,
-                                          uint32_t bars, uint32_t tmem, volatile int* abort)
+__device__ __forceinline__ void sf_load_group(uint4 (&v)[SF_WORDS], const SfGroup& c, const MxParams& p, int total,
+                                              int lane)
+{
+    if (c.item >= total) return;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        int64_t m = c.row0 + lane + 32 * j;
+        m = m < p.P ? m : p.P - 1;
+        // one 128-byte line per 8 lanes: the A scales are K-group-major
+        v[j] = mask_sf16(__ldg(reinterpret_cast<const uint4*>(p.a_sf + ((c.kb0 >> 2) * p.P + m) * 16)), 4 * c.kb0,
+                         p.a_chunks);
+    }
+#pragma unroll
+    for (int j = 0; j < 6; ++j) {
+        const uint8_t* base;
+        int row;
+        if (MODE == 0) {  // B rows 0..95 gate, 96..191 up
+            base = j < 3 ? p.b_sf0 : p.b_sf1;
+            row = c.w.nt * MX_HALF + lane + 32 * (j % 3);
+        } else {
+            base = p.b_sf0;
+            row = c.w.nt * MX_BN + lane + 32 * j;
+        }
+        const int64_t gw = (static_cast<int64_t>(c.w.e) * p.num_groups + (c.kb0 >> 2)) * p.b_rows + row;
+        v[4 + j] = row < p.b_rows ? mask_sf16(__ldg(reinterpret_cast<const uint4*>(base + gw * 16)), 4 * c.kb0,
+                                              p.b_chunks)
+                                  : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);  // padding rows
+    }
+}
+
+// Scale loader (warp 2, all lanes): writes each K block's words into the
+// shared slot it % SF_SLOTS, laid out [word][lane] (conflict-free), with the
+// next group's loads already in flight.  It issues no tcgen05 operation: a
+// tcgen05 wait also waits for the warp's outstanding global loads, so the
+// warps that write TMEM keep none.
+__device__ __forceinline__ bool sf_put(const uint4 (&v)[SF_WORDS], int i, int it, uint32_t sfs, uint32_t bars,
+                                       volatile int* abort)
+{
+    const int ss = it % SF_SLOTS;
+    if (!__all_sync(0xFFFFFFFFu,
+                    mbar_wait_bounded(bars + 8 * (MB_SSE + ss), ((it / SF_SLOTS) & 1) ^ 1, abort, MX_WAIT_NS)))
+        return false;
+    const int lane = threadIdx.x & 31;
+    const uint32_t slot = sfs + ss * (SF_WORDS * 32 * 4) + lane * 4;
+#pragma unroll
+    for (int j = 0; j < SF_WORDS; ++j) {
+        const uint32_t w = i == 0 ? v[j].x : i == 1 ? v[j].y : i == 2 ? v[j].z : v[j].w;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(slot + j * 128), "r"(w) : "memory");
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + 8 * (MB_SSF + ss));
+    return true;
+}
+
+// Put the K blocks of one group (at most four; fewer at an item's end).
+__device__ __forceinline__ bool sf_put_group(const uint4 (&v)[SF_WORDS], int nk, int& it, uint32_t sfs,
+                                             uint32_t bars, volatile int* abort)
+{
+    for (int i = 0; i < nk; ++i, ++it)
+        if (!sf_put(v, i, it, sfs, bars, abort)) return false;
+    return true;
+}
+
+template <int MODE>
+__device__ __forceinline__ void mx_sf_loader(const MxParams& p, const int* seg, const int* ipre, int total,
+                                             uint32_t sfs, uint32_t bars, volatile int* abort)
+{
+    const int lane = threadIdx.x & 31;
+    const int n_items = static_cast<int>(blockIdx.x) < total ? (total - 1 - static_cast<int>(blockIdx.x)) /
+                                                                      static_cast<int>(gridDim.x) + 1
+                                                                : 0;
+    const int steps = n_items * p.num_kb;
+    if (steps == 0) return;
+    SfGroup c;
+    c.item = blockIdx.x;
+    c.kb0 = 0;
+    c.w = mx_decode(seg, ipre, p.E, c.item);
+    c.row0 = seg[c.w.e] + c.w.mt * MX_BM;
+    uint4 g0[SF_WORDS], g1[SF_WORDS];
+    int n0 = min(4, p.num_kb - c.kb0);
+    sf_load_group<MODE>(g0, c, p, total, lane);
+    sf_group_next(c, p, seg, ipre, total);
+    int n1 = min(4, p.num_kb - c.kb0);
+    sf_load_group<MODE>(g1, c, p, total, lane);
+    sf_group_next(c, p, seg, ipre, total);
+    int it = 0;
+    while (it < steps) {
+        // put group 0, refill it with the group after next; then group 1
+        if (!sf_put_group(g0, n0, it, sfs, bars, abort)) return;
+        n0 = min(4, p.num_kb - c.kb0);
+        sf_load_group<MODE>(g0, c, p, total, lane);
+        sf_group_next(c, p, seg, ipre, total);
+        if (it >= steps) break;
+        if (!sf_put_group(g1, n1, it, sfs, bars, abort)) return;
+        n1 = min(4, p.num_kb - c.kb0);
+        sf_load_group<MODE>(g1, c, p, total, lane);
+        sf_group_next(c, p, seg, ipre, total);
+    }
+}
+
+// Scale writers (warps 8..11, all lanes): per K block, copy the shared slot
+// into TMEM lane 32q + t of the TMEM slot (columns 0..3 A rows t + 32j,
+// columns 8..13 B rows t + 32j) once the MMAs that read its previous
+// contents are done, then hand it to the MMA issuer.
+__device__ __forceinline__ void mx_sf_writer(int steps, uint32_t sfs, uint32_t bars, uint32_t tmem,
+                                             volatile int* abort)
 {
     const int lane = threadIdx.x & 31;
     const int q = (threadIdx.x >> 5) & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const bool a_aligned = (p.a_sf_stride & 3) == 0;
-    const bool b_aligned = (p.b_sf_stride & 3) == 0;
-    int it = 0;
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        const MxItem w = mx_decode(seg, ipre, p.E, item);
-        const int row0 = seg[w.e] + w.mt * MX_BM;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-            const int ss = it % SF_SLOTS;
-            uint32_t v[8];
+    for (int it = 0; it < steps; ++it) {
+        const int ss = it % SF_SLOTS;
+        const uint32_t ph = (it / SF_SLOTS) & 1;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SSF + ss), ph, abort, MX_WAIT_NS))) return;
+        uint32_t v[SF_WORDS];
+        const uint32_t slot = sfs + ss * (SF_WORDS * 32 * 4) + lane * 4;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                int64_t m = row0 + lane + 32 * c;
-                m = m < p.P ? m : p.P - 1;
-                v[c] = load_sf4(p.a_sf + m * p.a_sf_stride, 4 * kb, p.a_chunks, a_aligned);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int n = lane + 32 * c;  // row of the B tile
-                const uint8_t* base;
-                int row;
-                if (MODE == 0) {
-                    base = n < 64 ? p.b_sf0 : p.b_sf1;
-                    row = w.nt * 64 + (n & 63);
-                } else {
-                    base = p.b_sf0;
-                    row = w.nt * 128 + n;
-                }
-                v[4 + c] = row < p.b_rows
-                               ? load_sf4(base + (static_cast<int64_t>(w.e) * p.b_rows + row) * p.b_sf_stride, 4 * kb,
-                                          p.b_chunks, b_aligned)
-                               : 0x7F7F7F7Fu;  // padding rows: zero weights, unit scales
-            }
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SFE + ss), ((it / SF_SLOTS) & 1) ^ 1, abort,
-                                                            MX_WAIT_NS)))
-                return;
-            tc_fence_after();
-            tmem_st32x8(lane_base + SF_COL + ss * 8, v);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars + 8 * (MB_SFF + ss));
-        }
+        for (int j = 0; j < SF_WORDS; ++j) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[j]) : "r"(slot + j * 128) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * (MB_SSE + ss));
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SFE + ss), ph ^ 1, abort, MX_WAIT_NS)))
+            return;
+        tc_fence_after();
+        const uint32_t a[8] = {v[0], v[1], v[2], v[3], 0u, 0u, 0u, 0u};
+        const uint32_t b[8] = {v[4], v[5], v[6], v[7], v[8], v[9], 0u, 0u};
+        const uint32_t col = lane_base + SF_COL + ss * SF_SLOT_COLS;
+        tmem_st32x8(col, a);
+        tmem_st32x8(col + 8, b);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * (MB_SFF + ss));
     }
 }
 
 // MMA issuer (one lane): per item, wait until the accumulator buffer of the
 // item's parity is drained; per K block, wait for the operand stage and the
-// scale slot, issue four N = 128, K = 32 block-scaled MMAs (chunk j reads
+// scale slot, issue four N = 192, K = 32 block-scaled MMAs (chunk j reads
 // byte j of the scale columns), and commit so that the stage and the slot are
 // released when those MMAs are done; after the item's last K block, commit
 // the accumulator to the epilogue.
@@ -313,13 +435,13 @@ __device__ __forceinline__ void mx_mma(const MxParams& p, const int* seg, const 
             {
                 const uint32_t a_addr = sbase + s * MX_STAGE;
                 const uint32_t b_addr = a_addr + MX_A_TILE;
-                const uint32_t d = tmem + b * 128;
-                const uint32_t sfa = tmem + SF_COL + ss * 8;
-                const uint32_t sfb = sfa + 4;
+                const uint32_t d = tmem + b * MX_BN;
+                const uint32_t sfa = tmem + SF_COL + ss * SF_SLOT_COLS;
+                const uint32_t sfb = sfa + 8;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     mma_mx(d, sw128_kmajor_desc(a_addr + j * 32), sw128_kmajor_desc(b_addr + j * 32),
-                           idesc_mx(128, 128, static_cast<uint32_t>(j)), sfa | (static_cast<uint32_t>(j) << 30),
+                           idesc_mx(MX_BM, MX_BN, static_cast<uint32_t>(j)), sfa | (static_cast<uint32_t>(j) << 30),
                            sfb | (static_cast<uint32_t>(j) << 30), (kb > 0 || j > 0) ? 1u : 0u);
                 mma_commit(bars + 8 * (MB_EMPTY + s));
                 mma_commit(bars + 8 * (MB_SFE + ss));
@@ -348,10 +470,12 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 }
 
 // Epilogue (warps 4..7): thread = one row of the tile (TMEM lane 32q + lane).
-//   gate/up: columns [0,64) hold g, [64,128) u of intermediate columns
-//            nt*64 .. nt*64+63; h = SiLU(g) * u; each 32-column half is one
+//   gate/up: columns [0,96) hold g, [96,192) u of intermediate columns
+//            nt*96 .. nt*96+95; h = SiLU(g) * u; each 32 columns are one
 //            MX block of the intermediate row: scale byte and 32 codes.
-//   down:    y[pair, nt*128 + c] = topk_w[pair] * acc[c] for c < 128.
+//   down:    y[pair, nt*192 + c] = topk_w[pair] * acc[c] for c < 192.
+// The accumulator is released after its last TMEM load, before the last
+// block's arithmetic and stores.
 template <int MODE>
 __device__ __forceinline__ void mx_epilogue(const MxParams& p, const int* seg, const int* ipre, int total,
                                             uint32_t bars, uint32_t tmem, volatile int* abort)
@@ -365,25 +489,27 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const int* seg, c
         const int b = nitem & 1;
         const int r = seg[w.e] + w.mt * MX_BM + q * 32 + lane;
         const bool valid = r < seg[w.e + 1];
+        int pair = -1;
+        if (MODE == 1 && valid) pair = __ldg(p.sorted_pairs + r);  // in flight during the wait
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_AF + b), (nitem >> 1) & 1, abort, MX_WAIT_NS)))
             return;
         tc_fence_after();
-        const uint32_t col = lane_base + b * 128;
+        const uint32_t col = lane_base + b * MX_BN;
         if (MODE == 0) {
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            for (int blk = 0; blk < MX_HALF / 32; ++blk) {
                 uint32_t g[32], u[32];
                 __syncwarp();  // the loads are warp-collective
-                tmem_ld32_issue(col + half * 32, g);
+                tmem_ld32_issue(col + blk * 32, g);
                 tmem_ld_wait(g);
-                tmem_ld32_issue(col + 64 + half * 32, u);
+                tmem_ld32_issue(col + MX_HALF + blk * 32, u);
                 tmem_ld_wait(u);
-                if (half == 1) {
+                if (blk == MX_HALF / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars + 8 * (MB_AE + b));
                 }
-                const int c0 = w.nt * 64 + half * 32;  // intermediate column of this block
+                const int c0 = w.nt * MX_HALF + blk * 32;  // intermediate column of this block
                 if (!valid || c0 >= p.I) continue;
                 float h[32];
                 float amax = 0.0f;
@@ -411,33 +537,29 @@ __device__ __forceinline__ void mx_epilogue(const MxParams& p, const int* seg, c
                 }
                 reinterpret_cast<uint4*>(dst)[0] = o0;
                 reinterpret_cast<uint4*>(dst)[1] = o1;
-                p.h_scales[static_cast<int64_t>(r) * (p.Ip / 32) + c0 / 32] = sc;
+                p.h_scales[((static_cast<int64_t>(c0) >> 9) * p.P + r) * 16 + ((c0 >> 5) & 15)] = sc;
             }
         } else {
-            int pair = -1;
             float wt = 0.f;
-            if (valid) {
-                pair = __ldg(p.sorted_pairs + r);
-                if (pair < 0 || pair >= p.P) {
-                    atomicOr(p.status, kDevBadPair);
-                    pair = -1;
-                } else {
-                    wt = __ldg(p.topk_w + pair);
-                }
+            if (pair >= p.P || (valid && pair < 0)) {
+                atomicOr(p.status, kDevBadPair);
+                pair = -1;
+            } else if (pair >= 0) {
+                wt = __ldg(p.topk_w + pair);
             }
-            float* dst = pair >= 0 ? p.y + static_cast<int64_t>(pair) * p.H + w.nt * 128 : nullptr;
+            float* dst = pair >= 0 ? p.y + static_cast<int64_t>(pair) * p.H + w.nt * MX_BN : nullptr;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < MX_BN / 32; ++c) {
                 uint32_t v[32];
                 __syncwarp();
                 tmem_ld32_issue(col + c * 32, v);
                 tmem_ld_wait(v);
-                if (c == 3) {
+                if (c == MX_BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars + 8 * (MB_AE + b));
                 }
-                if (!dst || w.nt * 128 + c * 32 >= p.H) continue;
+                if (!dst || w.nt * MX_BN + c * 32 >= p.H) continue;
                 float4* g4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
@@ -471,8 +593,10 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
             mbar_init(bars + 8 * (MB_EMPTY + s), 1);  // MMA commit
         }
         for (int s = 0; s < SF_SLOTS; ++s) {
-            mbar_init(bars + 8 * (MB_SFF + s), 4);    // four stager warps
+            mbar_init(bars + 8 * (MB_SFF + s), 4);    // four writer warps
             mbar_init(bars + 8 * (MB_SFE + s), 1);    // MMA commit
+            mbar_init(bars + 8 * (MB_SSF + s), 1);    // the loader warp
+            mbar_init(bars + 8 * (MB_SSE + s), 4);    // four writer warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars + 8 * (MB_AF + b), 1);     // MMA commit
@@ -521,10 +645,14 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
             else if (warp == 1) mx_mma(p, seg, ipre, total, sbase, bars, tmem, abort);
             else if (warp == 3) mx_producer_a(&tmA, p, seg, ipre, total, sbase, bars, abort);
         }
+        if (warp == 2) mx_sf_loader<MODE>(p, seg, ipre, total, sbase + MX_OFF_SFS, bars, abort);
     } else if (warp < 8) {
         mx_epilogue<MODE>(p, seg, ipre, total, bars, tmem, abort);
     } else {
-        mx_stager<MODE>(p, seg, ipre, total, bars, tmem, abort);
+        const int n_items = static_cast<int>(blockIdx.x) < total
+                                ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                : 0;
+        mx_sf_writer(n_items * p.num_kb, sbase + MX_OFF_SFS, bars, tmem, abort);
     }
 
     tc_fence_before();
@@ -537,7 +665,9 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
 }
 
 // Gather: one warp per sorted row r < P_valid copies the token's code row
-// and its H/32 scale bytes into expert order.
+// and its H/32 scale bytes into expert order, the scales K-group-major
+// ([ceil(H/512)][P][16]) so that the scale loader reads 32 rows' group with
+// one coalesced request.
 __global__ void __launch_bounds__(256) gather_mx_kernel(const uint8_t* __restrict__ codes,
                                                         const uint8_t* __restrict__ act_scales, int H, int k,
                                                         const int32_t* __restrict__ sorted_pairs,
@@ -569,9 +699,40 @@ __global__ void __launch_bounds__(256) gather_mx_kernel(const uint8_t* __restric
             for (int u = 0; u < 4; ++u)
                 if (c0 + 32 * u < n16) dst[c0 + 32 * u] = v[u];
         }
+        // scale words K-group-major: group g of row r at (g * P + r) * 16
         const uint32_t* ss = reinterpret_cast<const uint32_t*>(act_scales + t * (H / 32));
-        uint32_t* sd = reinterpret_cast<uint32_t*>(sa_sorted + r * (H / 32));
-        for (int c = lane; c < n4; c += 32) sd[c] = __ldg(ss + c);
+        for (int c = lane; c < n4; c += 32)
+            reinterpret_cast<uint32_t*>(sa_sorted + ((c >> 2) * P + r) * 16)[c & 3] = __ldg(ss + c);
+    }
+}
+
+// Weight scales [E, R, K/32] -> K-group-major [E][ceil(K/512)][R][16]: one
+// thread per 16-byte output word; chunks at or past K/32 are written as 127.
+__global__ void __launch_bounds__(256) pack_scales_kernel(const uint8_t* __restrict__ src, int64_t E, int R, int K,
+                                                          uint8_t* __restrict__ dst)
+{
+    const int C = K / 32;
+    const int G = (K + 511) / 512;
+    const int64_t n = E * G * R;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int r = static_cast<int>(i % R);
+        const int64_t eg = i / R;
+        const int g = static_cast<int>(eg % G);
+        const int64_t e = eg / G;
+        const uint8_t* row = src + (e * R + r) * C;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int c = 16 * g + 4 * q + b;
+                v |= static_cast<uint32_t>(c < C ? __ldg(row + c) : 0x7F) << (8 * b);
+            }
+            w[q] = v;
+        }
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -595,6 +756,20 @@ cudaError_t run_mx(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
 
 }  // namespace
 
+int mx_scale_groups(int K) { return (K + 511) / 512; }
+
+cudaError_t launch_pack_mx_scales(const uint8_t* src, int64_t E, int R, int K, uint8_t* dst, cudaStream_t s)
+{
+    const int64_t n = E * mx_scale_groups(K) * R;
+    if (n == 0) return cudaSuccess;
+    DeviceInfo di;
+    if (!device_info(&di)) return cudaErrorUnknown;
+    const int64_t want = ceil_div64(n, 256);
+    const int64_t cap = static_cast<int64_t>(di.sm_count) * 8;
+    pack_scales_kernel<<<static_cast<int>(want < cap ? want : cap), 256, 0, s>>>(src, E, R, K, dst);
+    return cudaGetLastError();
+}
+
 size_t ffn_mx_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
                                size_t* off_sh)
 {
@@ -604,11 +779,11 @@ size_t ffn_mx_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, si
     *off_a = o;
     o = align_up(o + static_cast<size_t>(P) * H, 256);
     *off_sa = o;
-    o = align_up(o + static_cast<size_t>(P) * (H / 32), 256);
+    o = align_up(o + static_cast<size_t>(P) * mx_scale_groups(H) * 16, 256);
     *off_h = o;
     o = align_up(o + static_cast<size_t>(P) * Ip, 256);
     *off_sh = o;
-    o = align_up(o + static_cast<size_t>(P) * (Ip / 32), 256);
+    o = align_up(o + static_cast<size_t>(P) * mx_scale_groups(static_cast<int>(Ip)) * 16, 256);
     return o;
 }
 
@@ -644,8 +819,8 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
     }
 
     // 2. tensor maps: activations and intermediate [rows, K] with 128-row
-    // boxes; gate/up weights with 64-row boxes (64 gate + 64 up rows per
-    // tile), down weights with 128-row boxes.  The intermediate's map is I
+    // boxes; gate/up weights with 96-row boxes (96 gate + 96 up rows per
+    // tile), down weights with 192-row boxes.  The intermediate's map is I
     // wide over rows of Ip bytes, so the padding columns of the last K block
     // read as zero.
     CUtensorMap tmA1, tmG, tmU, tmA2, tmD;
@@ -659,10 +834,10 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
         const uint64_t dD[3] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H), static_cast<uint64_t>(E)};
         const uint64_t sD[2] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H) * I};
         if (!a.down_only && (!make_tmap_u8(&tmA1, a.a_sorted, 2, dA, sA, 128) ||
-                             !make_tmap_u8(&tmG, a.w_gate, 3, dW, sW, 64) ||
-                             !make_tmap_u8(&tmU, a.w_up, 3, dW, sW, 64)))
+                             !make_tmap_u8(&tmG, a.w_gate, 3, dW, sW, MX_HALF) ||
+                             !make_tmap_u8(&tmU, a.w_up, 3, dW, sW, MX_HALF)))
             return cudaErrorNotSupported;
-        if (!make_tmap_u8(&tmA2, a.h_codes, 2, dH, sH, 128) || !make_tmap_u8(&tmD, a.w_down, 3, dD, sD, 128))
+        if (!make_tmap_u8(&tmA2, a.h_codes, 2, dH, sH, 128) || !make_tmap_u8(&tmD, a.w_down, 3, dD, sD, MX_BN))
             return cudaErrorNotSupported;
     }
     const int grid = di.sm_count;
@@ -671,16 +846,15 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
     MxParams g{};
     g.E = E;
     g.num_kb = (H + MX_BK - 1) / MX_BK;
-    g.n_tiles = (I + 63) / 64;
+    g.num_groups = mx_scale_groups(H);
+    g.n_tiles = (I + MX_HALF - 1) / MX_HALF;
     g.P = P;
     g.offsets = a.expert_offsets;
     g.a_sf = a.sa_sorted;
-    g.a_sf_stride = H / 32;
     g.a_chunks = H / 32;
     g.b_sf0 = a.s_gate;
     g.b_sf1 = a.s_up;
     g.b_rows = I;
-    g.b_sf_stride = H / 32;
     g.b_chunks = H / 32;
     g.h_codes = a.h_codes;
     g.h_scales = a.h_scales;
@@ -697,14 +871,13 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
     // 4. down GEMM with the routing-weighted row epilogue
     MxParams d = g;
     d.num_kb = Ip / MX_BK;
-    d.n_tiles = (H + 127) / 128;
+    d.num_groups = mx_scale_groups(Ip);
+    d.n_tiles = (H + MX_BN - 1) / MX_BN;
     d.a_sf = a.h_scales;
-    d.a_sf_stride = Ip / 32;
     d.a_chunks = I / 32;
     d.b_sf0 = a.s_down;
     d.b_sf1 = a.s_down;
     d.b_rows = H;
-    d.b_sf_stride = I / 32;
     d.b_chunks = I / 32;
     if ((err = mx_stage_mark(a, 2, s)) != cudaSuccess) return err;
     if ((err = run_mx<1>(tmA2, tmD, tmD, d, grid, s)) != cudaSuccess) return err;

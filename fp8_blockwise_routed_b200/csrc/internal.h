@@ -162,20 +162,26 @@ struct FfnMxArgs {
     int E;
     int I;
     const uint8_t* w_gate;
-    const uint8_t* s_gate;  // [E, I, H/32]
+    const uint8_t* s_gate;  // packed [E][ceil(H/512)][I][16] (moe_mx_pack_scales)
     const uint8_t* w_up;
     const uint8_t* s_up;
     const uint8_t* w_down;
-    const uint8_t* s_down;  // [E, H, I/32]
+    const uint8_t* s_down;  // packed [E][ceil(I/512)][H][16]
     float* y;               // [T, k, H]
     int* status;
     uint8_t* a_sorted;      // [P, H] codes in expert order
-    uint8_t* sa_sorted;     // [P, H/32] scale bytes in expert order
+    uint8_t* sa_sorted;     // [ceil(H/512)][P][16] scale bytes in expert order, K-group-major
     uint8_t* h_codes;       // [P, Ip]
-    uint8_t* h_scales;      // [P, Ip/32]
+    uint8_t* h_scales;      // [ceil(Ip/512)][P][16], the same layout
     void* const* stage_events;
     int down_only;          // 1: h_codes / h_scales are inputs; only the down GEMM runs
 };
+// Groups of four K blocks (512 values) of a K-wide MX operand: its scales sit
+// in the workspace as [groups][rows][16 bytes].
+int mx_scale_groups(int K);
+// MX weight scales [E, R, K/32] -> [E][mx_scale_groups(K)][R][16] (padding
+// chunks 127).
+cudaError_t launch_pack_mx_scales(const uint8_t* src, int64_t E, int R, int K, uint8_t* dst, cudaStream_t s);
 size_t ffn_mx_workspace_layout(int64_t T, int H, int I, int k, size_t* off_a, size_t* off_sa, size_t* off_h,
                                size_t* off_sh);
 cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s);

@@ -304,8 +304,10 @@ MOE_API int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64
  *
  *   codes, act_scales      [T, H] uint8, [T, H/32] uint8  (moe_quant_act_mx output)
  *   topk_ids, topk_w, expert_offsets, sorted_pairs   as moe_grouped_ffn
- *   w_gate, w_up           [E, I, H] uint8 E4M3;  s_gate, s_up [E, I, H/32] uint8 UE8M0
- *   w_down                 [E, H, I] uint8 E4M3;  s_down       [E, H, I/32] uint8 UE8M0
+ *   w_gate, w_up           [E, I, H] uint8 E4M3
+ *   s_gate, s_up           UE8M0 bytes of [E, I, H/32], packed by moe_mx_pack_scales
+ *   w_down                 [E, H, I] uint8 E4M3
+ *   s_down                 UE8M0 bytes of [E, H, I/32], packed by moe_mx_pack_scales
  *   y                      [T, top_k, H] FP32, written (valid slots only)
  *   ws, ws_bytes           scratch of at least moe_ffn_mx_workspace_bytes(T, H, I, E, top_k)
  *   stage_events           as moe_grouped_ffn
@@ -315,6 +317,19 @@ MOE_API int moe_grouped_ffn(const uint8_t* codes, const float* act_scales, int64
  * and code bytes 0x7F/0xFF in the weights are outside the contract.
  * Errors as moe_grouped_ffn.
  * ------------------------------------------------------------------------- */
+/* moe_mx_pack_scales -- weight scale bytes from the checkpoint layout
+ * src [E, R, K/32] (row r's scale of columns 32c..32c+31 at byte c) into the
+ * layout the MX FFN reads: dst [E][G][R][16], G = ceil(K/512), where byte
+ * (e, g, r, b) holds chunk 16g + b of row r (127, i.e. 2^0, for chunks at or
+ * past K/32).  Each 16-byte word covers four K blocks of one row, and 32
+ * consecutive rows' words are contiguous: the kernel loads a tile's scales
+ * for four K blocks with one coalesced request per lane.  A one-time
+ * transformation of static weights (no counterpart on the pages).
+ *   src  device, read;  dst device, moe_mx_packed_scales_bytes(E, R, K) bytes, written
+ * Limits: E >= 0, R >= 1, K % 32 == 0, K >= 32.  Errors: MOE_ERR_INVALID_ARG,
+ * MOE_ERR_ALIGNMENT (dst not 16-byte aligned), MOE_ERR_CUDA. */
+MOE_API size_t moe_mx_packed_scales_bytes(int64_t E, int R, int K);
+MOE_API int moe_mx_pack_scales(const uint8_t* src, int64_t E, int R, int K, uint8_t* dst, void* stream);
 MOE_API size_t moe_ffn_mx_workspace_bytes(int64_t T, int H, int I, int E, int top_k);
 MOE_API int moe_grouped_ffn_mx(const uint8_t* codes, const uint8_t* act_scales, int64_t T, int H,
                                const int32_t* topk_ids, const float* topk_w, int top_k,
@@ -552,15 +567,17 @@ MOE_API int moe_debug_grouped_down(const uint8_t* h_codes, const float* h_scales
 /* moe_ffn_mx_intermediate: device pointers into a workspace last used by
  * moe_grouped_ffn_mx with the same (T, H, I, top_k): the MX intermediate
  * codes [T*top_k, Ip] (columns I..Ip-1 unspecified, Ip = ceil(I/128)*128)
- * and scale bytes [T*top_k, Ip/32] (bytes I/32.. unspecified), rows in
- * expert order.  Host arithmetic only. */
+ * and scale bytes [G][T*top_k][16], G = ceil(Ip/512): the scale of row r,
+ * columns 32c..32c+31 is byte (c/16 * T*top_k + r) * 16 + c%16 (chunks c >=
+ * I/32 unspecified); rows in expert order.  Host arithmetic only. */
 MOE_API int moe_ffn_mx_intermediate(const void* ws, int64_t T, int H, int I, int top_k,
                                     const uint8_t** h_codes, const uint8_t** h_scales);
 
 /* moe_debug_grouped_down_mx: the down GEMM of moe_grouped_ffn_mx alone, on
  * an intermediate the caller supplies in the layout moe_ffn_mx_intermediate
- * describes (h_codes [T*top_k, Ip], h_scales [T*top_k, Ip/32], expert
- * order).  Writes y as moe_grouped_ffn_mx's down stage does (same kernel).
+ * describes (h_codes [T*top_k, Ip], h_scales [G][T*top_k][16], expert
+ * order; scale bytes of chunks at or past I/32 are not used), with s_down
+ * packed by moe_mx_pack_scales.  Writes y as moe_grouped_ffn_mx's down stage does (same kernel).
  * Workspace: at least moe_combine_workspace_bytes().  Limits and errors as
  * moe_grouped_ffn_mx. */
 MOE_API int moe_debug_grouped_down_mx(const uint8_t* h_codes, const uint8_t* h_scales, int64_t T, int H,

@@ -99,6 +99,32 @@ def _mx_dequant(codes_u8, scale_bytes):
     return v * sc.repeat_interleave(32, dim=-1)[..., : v.shape[-1]]
 
 
+_packed: dict = {}
+
+
+def packed(d):
+    """The weight scales of d packed by moe_mx_pack_scales (once per tensor)."""
+    key = tuple(d[n].data_ptr() for n in ("s_gate", "s_up", "s_down"))
+    if key not in _packed:
+        _packed.clear()
+        _packed[key] = {n: fm.moe_mx_pack_scales(d[n]) for n in ("s_gate", "s_up", "s_down")}
+    return _packed[key]
+
+
+def test_mx_pack_scales():
+    """The packed layout is a pure permutation of the checkpoint bytes (plus
+    127 padding), on even and ragged K/32."""
+    g = torch.Generator().manual_seed(5)
+    for E, R, K in ((3, 70, 5120), (2, 33, 192), (1, 5, 32), (4, 192, 1536), (2, 8, 2080)):
+        src = torch.randint(0, 255, (E, R, K // 32), generator=g, dtype=torch.uint8)
+        dst = fm.moe_mx_pack_scales(src.cuda()).cpu().numpy()
+        G = (K + 511) // 512
+        want = np.full((E, R, G * 16), 127, np.uint8)
+        want[:, :, : K // 32] = src.numpy()
+        want = want.reshape(E, R, G, 16).transpose(0, 2, 1, 3)
+        assert np.array_equal(dst, want)
+
+
 def run_mx_layer(wl, d, rs=None):
     """Route (moe_route), quantise (moe_quant_act_mx), experts
     (moe_grouped_ffn_mx), combine (moe_combine) on CUDA tensors ``d``."""
@@ -119,8 +145,9 @@ def run_mx_layer(wl, d, rs=None):
     fm.moe_quant_act_mx(x, codes, scales)
     ws = torch.zeros((fm.moe_ffn_mx_workspace_bytes(T, H, I, E, k),), dtype=torch.uint8, device=dev)
     y = torch.zeros((T, k, H), dtype=torch.float32, device=dev)
-    fm.moe_grouped_ffn_mx(codes, scales, ids, tw, off, sp, d["w_gate"], d["s_gate"], d["w_up"], d["s_up"],
-                          d["w_down"], d["s_down"], y, ws)
+    pk = packed(d)
+    fm.moe_grouped_ffn_mx(codes, scales, ids, tw, off, sp, d["w_gate"], pk["s_gate"], d["w_up"], pk["s_up"],
+                          d["w_down"], pk["s_down"], y, ws)
     out = torch.empty((T, H), dtype=torch.float32, device=dev)
     cws = torch.zeros((fm.moe_combine_workspace_bytes(),), dtype=torch.uint8, device=dev)
     fm.moe_combine(y, ids, E, rs, out, None, cws)
@@ -137,8 +164,10 @@ def _gpu_h_by_pair(g, wl, T):
     sp = g["sorted"][:P].cpu().numpy()
     gc = np.zeros((T * k, I), np.uint8)
     gs = np.zeros((T * k, I // 32), np.uint8)
+    G = hs.shape[0]
+    rows = hs.permute(1, 0, 2).reshape(T * k, G * 16)  # [P, chunk]
     gc[sp] = hc[:P, :I].cpu().numpy()
-    gs[sp] = hs[:P, : I // 32].cpu().numpy()
+    gs[sp] = rows[:P, : I // 32].cpu().numpy()
     return gc.reshape(T, k, I), gs.reshape(T, k, I // 32)
 
 
@@ -272,18 +301,22 @@ def test_mx_layer_matches_oracle(name):
     # literal tolerance with no allowance
     k, I, H = wl.k, wl.I, wl.H
     Ip = (I + 127) // 128 * 128
+    G = (Ip + 511) // 512
+    SI = G * 16
     hc = np.zeros((T, k, Ip), np.uint8)
-    hs = np.full((T, k, Ip // 32), 127, np.uint8)
+    hs = np.full((T, k, SI), 0xFF, np.uint8)  # bytes past I/32 must not be used
+    hs[:, :, : I // 32] = 127
     hc[toks, :, :I] = ref["h_codes"]
     hs[toks, :, : I // 32] = ref["h_scales"]
     hc_s = np.zeros((T * k, Ip), np.uint8)
-    hs_s = np.full((T * k, Ip // 32), 127, np.uint8)
+    hs_s = np.full((T * k, SI), 0xFF, np.uint8)
     hc_s[:P] = hc.reshape(T * k, Ip)[sp_o[:P]]
-    hs_s[:P] = hs.reshape(T * k, Ip // 32)[sp_o[:P]]
+    hs_s[:P] = hs.reshape(T * k, SI)[sp_o[:P]]
     y = torch.zeros((T, k, H), dtype=torch.float32, device="cuda")
     cws = torch.zeros((fm.moe_combine_workspace_bytes(),), dtype=torch.uint8, device="cuda")
-    fm.moe_debug_grouped_down_mx(torch.from_numpy(hc_s).cuda(), torch.from_numpy(hs_s).cuda(), g["w"],
-                                 g["offsets"], g["sorted"][: T * k], d["w_down"], d["s_down"], y, cws)
+    hs_g = np.ascontiguousarray(hs_s.reshape(T * k, G, 16).transpose(1, 0, 2))  # [G, P, 16]
+    fm.moe_debug_grouped_down_mx(torch.from_numpy(hc_s).cuda(), torch.from_numpy(hs_g).cuda(), g["w"],
+                                 g["offsets"], g["sorted"][: T * k], d["w_down"], packed(d)["s_down"], y, cws)
     torch.cuda.synchronize()
     assert fm.moe_get_device_status(cws) == 0
     out = torch.empty((T, H), dtype=torch.float32, device="cuda")
