@@ -193,10 +193,11 @@ def gateup_alg_bytes(wl, active: int, P: int) -> float:
             + wl.T * wl.H + 4.0 * wl.T * wl.GH + P * wl.Ip + 4.0 * P * wl.GI)
 
 
-def cpu_baseline(wl, d, budget_tokens: int | None = None, seconds: float = 20.0):
+def cpu_baseline(wl, d, budget_tokens: int | None = None, seconds: float = 20.0, mx: bool = False):
     """The oracle as it stands (plain C, FP64, OpenMP) on a seeded token
     sample of the same workload (sized to about ``seconds`` of work), timed
-    on the host.  Returns tokens/s."""
+    on the host; mx: the MXFP8 variant's oracle on MX inputs.  Returns
+    tokens/s."""
     import oracle
 
     g = mi.generator(0, "cpu_baseline", "cpu")
@@ -208,7 +209,7 @@ def cpu_baseline(wl, d, budget_tokens: int | None = None, seconds: float = 20.0)
     def run(n):
         toks = perm[:n].sort().values
         t0 = time.perf_counter()
-        oracle.moe_layer(xs[toks], ls[toks], wl.k, *W, wl.routed_scaling)
+        (oracle.mx_moe_layer if mx else oracle.moe_layer)(xs[toks], ls[toks], wl.k, *W, wl.routed_scaling)
         return time.perf_counter() - t0
 
     if budget_tokens:
@@ -218,8 +219,8 @@ def cpu_baseline(wl, d, budget_tokens: int | None = None, seconds: float = 20.0)
         n = max(probe, min(wl.T, int(seconds * probe / max(run(probe), 1e-6))))
     dt = run(n)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n} seeded tokens of the {wl.name} workload (quantise, route, FFN, combine), "
-                      f"{dt:.1f} s"}
+            "sample": f"{n} seeded tokens of the {wl.name} workload ({'MX ' if mx else ''}quantise, route, FFN, "
+                      f"combine), {dt:.1f} s"}
 
 
 def run_reference(args, wl):
@@ -375,6 +376,58 @@ def measure_workload(wl, steps: int, warmup: int, seed: int, pk, with_cpu: bool)
         res["cpu_oracle"] = cpu_baseline(wl, d, seconds=3.0)
     plan.close()
     del plan, layer, d, x_in, lg_in, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_workload_mx(wl, steps: int, warmup: int, seed: int, pk, with_cpu: bool):
+    """The MXFP8 variant of the layer on one workload (the same FP32 weight
+    draws, stored as MX E4M3 with UE8M0 scales per 32 values): device time per
+    step of RoutedMoEMX.forward (4 ABI calls, no graph), per-stage means, the
+    grouped GEMMs against the same roofline as the 128x128-block path, and
+    the MX oracle on a ~3 s token sample."""
+    import fp8_blockwise_routed_b200 as fm
+
+    d = mi.make_inputs_mx(wl, seed=seed, device="cuda")
+    layer = fm.RoutedMoEMX(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"], wl.k,
+                           wl.routed_scaling, wl.T)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for e in ev:
+        e.record()
+    for _ in range(warmup):
+        layer.forward(d["x"], d["logits"])
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for _ in range(steps):
+        layer.forward(d["x"], d["logits"])
+    t1.record(s)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    spans = {"quant_route": (0, 1), "gather": (1, 2), "gemm_gateup": (2, 3), "gemm_down": (3, 4),
+             "combine": (4, 5)}
+    acc = {n: [] for n in spans}
+    for _ in range(max(steps, 5)):
+        layer.forward(d["x"], d["logits"], stage_events=ev)
+        torch.cuda.synchronize()
+        for n, (a, b) in spans.items():
+            acc[n].append(ev[a].elapsed_time(ev[b]))
+    st = {n: statistics.mean(v) for n, v in acc.items()}
+    off = layer.offsets.cpu()
+    P = int(off[-1])
+    active = int(((off[1:] - off[:-1]) > 0).sum())
+    gemm_s = (st["gemm_gateup"] + st["gemm_down"]) / 1e3
+    flops = mi.flops_per_layer(wl, P)
+    roof = gemm_roofline_s(wl, P, active, pk)
+    res = {"format": "MXFP8 (E4M3, UE8M0 scale per 32 values)", "ms_per_step": ms,
+           "tokens_per_s": wl.T / (ms / 1e3), "stages_ms": st, "gemm_tflops": flops / gemm_s / 1e12,
+           "gemm_roofline_ms": roof * 1e3, "gemm_frac_roofline": roof / gemm_s, "pairs": P,
+           "active_experts": active, "device_status": layer.device_status()}
+    if with_cpu:
+        res["cpu_oracle"] = cpu_baseline(wl, d, seconds=3.0, mx=True)
+    del layer, d
     torch.cuda.empty_cache()
     return res
 
@@ -570,6 +623,9 @@ def main():
                 continue
             configs[name] = measure_workload(mi.WORKLOADS[name], args.steps, args.warmup, rank_seed(rank), pk,
                                              with_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+        configs[wl.name + "_mxfp8"] = measure_workload_mx(
+            wl, args.steps, args.warmup, rank_seed(rank), pk,
+            with_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
 
     if rank == 0:
         line = {

@@ -547,3 +547,62 @@ class RoutedMoE:
     def device_status(self) -> int:
         return (moe_get_device_status(self.ws_route) | moe_get_device_status(self.ws_ffn)
                 | moe_get_device_status(self.ws_comb))
+
+
+class RoutedMoEMX:
+    """One routed-expert layer of the MXFP8 variant: resident E4M3 weights
+    with UE8M0 scales per 32 values (packed once by moe_mx_pack_scales at
+    construction), buffers for up to `max_tokens` rows.  ``forward`` enqueues
+    moe_quant_act_mx, moe_route, moe_grouped_ffn_mx and moe_combine on the
+    current stream and returns the FP32 output rows."""
+
+    def __init__(self, w_gate, s_gate, w_up, s_up, w_down, s_down, top_k: int, routed_scaling: float,
+                 max_tokens: int):
+        self.E, self.I, self.H = w_gate.shape
+        self.w = (w_gate, moe_mx_pack_scales(s_gate), w_up, moe_mx_pack_scales(s_up), w_down,
+                  moe_mx_pack_scales(s_down))
+        self.k = int(top_k)
+        self.rs = float(routed_scaling)
+        self.max_tokens = int(max_tokens)
+        dev = w_gate.device
+        T, H, E, k = self.max_tokens, self.H, self.E, self.k
+        u8, i32, f32 = torch.uint8, torch.int32, torch.float32
+        self.codes = torch.empty((T, H), dtype=u8, device=dev)
+        self.scales = torch.empty((T, H // 32), dtype=u8, device=dev)
+        self.ids = torch.empty((T, k), dtype=i32, device=dev)
+        self.tw = torch.empty((T, k), dtype=f32, device=dev)
+        self.offsets = torch.empty((E + 1,), dtype=i32, device=dev)
+        self.sorted = torch.empty((max(T * k, 1),), dtype=i32, device=dev)
+        self.y = torch.empty((T, k, H), dtype=f32, device=dev)
+        self.out = torch.empty((T, H), dtype=f32, device=dev)
+        self.ws_route = torch.empty((moe_route_workspace_bytes(T, E, k),), dtype=u8, device=dev)
+        self.ws_ffn = torch.empty((moe_ffn_mx_workspace_bytes(T, H, self.I, E, k),), dtype=u8, device=dev)
+        self.ws_comb = torch.empty((moe_combine_workspace_bytes(),), dtype=u8, device=dev)
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, out_bf16: torch.Tensor | None = None,
+                stream=None, stage_events=None) -> torch.Tensor:
+        """stage_events: None, or 6 recorded torch.cuda.Events marking the
+        start of quantise + route, gather, gate/up, down, combine and the end."""
+        T = x.shape[0]
+        assert T <= self.max_tokens and x.shape[1] == self.H and logits.shape == (T, self.E)
+        codes, scales = self.codes[:T], self.scales[:T]
+        ids, tw, srt = self.ids[:T], self.tw[:T], self.sorted[: max(T * self.k, 1)]
+        y, out = self.y[:T], self.out[:T]
+        ev = stage_events
+        s = torch.cuda.current_stream() if stream is None else stream
+        if ev is not None:
+            ev[0].record(s)
+        moe_quant_act_mx(x, codes, scales, stream)
+        moe_route(logits, self.k, ids, tw, self.offsets, srt, self.ws_route, stream)
+        moe_grouped_ffn_mx(codes, scales, ids, tw, self.offsets, srt, *self.w, y, self.ws_ffn, stream,
+                           stage_events=None if ev is None else ev[1:5])
+        moe_combine(y, ids, self.E, self.rs, out, out_bf16, self.ws_comb, stream)
+        if ev is not None:
+            ev[5].record(s)
+        return out
+
+    def device_status(self) -> int:
+        return (moe_get_device_status(self.ws_route) | moe_get_device_status(self.ws_ffn)
+                | moe_get_device_status(self.ws_comb))
+
+
