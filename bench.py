@@ -432,21 +432,29 @@ def measure_workload_mx(wl, steps: int, warmup: int, seed: int, pk, with_cpu: bo
     return res
 
 
-def layer_only(wl, n: int):
+def layer_only(wl, n: int, mx: bool = False):
     """The layer of `wl` (seed 0) n times through moe_route_quant,
     moe_grouped_ffn and moe_combine, for profiler captures: each call launches
     route_topk, route_rank, route_scatter, gather_rows, grouped_gemm (gate/up),
-    grouped_gemm (down) and combine, in that order."""
+    grouped_gemm (down) and combine, in that order.  mx: the MXFP8 variant
+    (RoutedMoEMX): quant_mx, route_topk, route_rank, route_scatter, gather_mx,
+    grouped_mx (gate/up), grouped_mx (down), combine."""
     import fp8_blockwise_routed_b200 as fm
 
-    d = mi.make_inputs(wl, seed=0, device="cuda")
-    layer = fm.RoutedMoE(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"], wl.k,
-                         wl.routed_scaling, wl.T)
+    if mx:
+        d = mi.make_inputs_mx(wl, seed=0, device="cuda")
+        cls = fm.RoutedMoEMX
+    else:
+        d = mi.make_inputs(wl, seed=0, device="cuda")
+        cls = fm.RoutedMoE
+    layer = cls(d["w_gate"], d["s_gate"], d["w_up"], d["s_up"], d["w_down"], d["s_down"], wl.k,
+                wl.routed_scaling, wl.T)
     for _ in range(n):
         layer.forward(d["x"], d["logits"])
     torch.cuda.synchronize()
     off = layer.offsets.cpu()
-    print(json.dumps({"workload": wl.name, "calls": n, "device_status": layer.device_status(),
+    print(json.dumps({"workload": wl.name, "format": "mxfp8" if mx else "fp8 128x128 blocks", "calls": n,
+                      "device_status": layer.device_status(),
                       "pairs": int(off[-1]), "active_experts": int(((off[1:] - off[:-1]) > 0).sum())}))
 
 
@@ -470,11 +478,12 @@ def main():
     ap.add_argument("--layer-only", type=int, default=0, metavar="N",
                     help="run the workload's layer N times through the separate calls and exit "
                          "(the program profiler captures run)")
+    ap.add_argument("--mxfp8", action="store_true", help="with --layer-only: the MXFP8 variant's layer")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = mi.WORKLOADS[args.workload]
     if args.layer_only:
-        layer_only(wl, args.layer_only)
+        layer_only(wl, args.layer_only, mx=args.mxfp8)
         return
     if args.impl == "reference":
         run_reference(args, wl)
