@@ -421,7 +421,7 @@ __device__ __forceinline__ void mx_sf_writer(int steps, uint32_t sfs, uint32_t b
 __device__ __forceinline__ void mx_mma(const MxParams& p, const int* seg, const int* ipre, int total, uint32_t sbase,
                                        uint32_t bars, uint32_t tmem, volatile int* abort)
 {
-    int it = 0, nitem = 0, last_item = -1;
+    int it = 0, nitem = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x, ++nitem) {
         const int b = nitem & 1;
         if (!mbar_spin_bounded(bars + 8 * (MB_AE + b), ((nitem >> 1) & 1) ^ 1, abort, MX_WAIT_NS)) goto drain;
@@ -448,16 +448,15 @@ __device__ __forceinline__ void mx_mma(const MxParams& p, const int* seg, const 
             }
         }
         mma_commit(bars + 8 * (MB_AF + b));
-        last_item = nitem;
     }
     return;
 drain:
-    // wait for the MMAs already issued before TMEM is released
-    if (last_item >= 0 || it > 0) {
+    // wait for the MMAs already issued before TMEM is released: the last
+    // slot commit tracks every MMA this thread issued
+    if (it > 0) {
         volatile int no_abort = 0;
-        // every MMA issued so far is tracked by the last slot commit
         const int j = it - 1;
-        if (j >= 0) mbar_wait_bounded(bars + 8 * (MB_SFE + j % SF_SLOTS), (j / SF_SLOTS) & 1, &no_abort, MX_WAIT_NS / 4);
+        mbar_wait_bounded(bars + 8 * (MB_SFE + j % SF_SLOTS), (j / SF_SLOTS) & 1, &no_abort, MX_WAIT_NS / 4);
     }
 }
 
