@@ -22,9 +22,9 @@
 //
 // Warp roles (384 threads, one CTA per SM, persistent over work items ordered
 // expert-major, then n-tile, then m-tile):
-//   warp 0      weight TMA producer (one lane)
+//   warp 0      weight TMA producers (lanes 0, 1: one 96-row half each)
 //   warp 1      MMA issuer (one lane; also allocates TMEM)
-//   warp 3      activation TMA producer (one lane)
+//   warp 3      activation TMA producers (lanes 0, 1: one 64-row half each)
 //   warps 4..7  epilogue: warp w drains TMEM lanes 32*(w%4), once per item
 //   warp 2      scale loader (all lanes): the tile's A and B scale bytes of
 //               each K block from global memory into a shared ring, four K
@@ -177,10 +177,17 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 // ---------------------------------------------------------------- roles
 
+// Weight producers (warp 0, lanes 0 and 1) and activation producers (warp 3,
+// lanes 0 and 1): each lane loads one half of its operand's tile per K
+// block (gate or up rows, the first or second 96 down rows; the first or
+// second 64 activation rows), and a stage is full when all four halves have
+// landed.  The TMA unit serves each issuing thread's requests one after
+// another, about 25 bytes per clock per thread (measured), so one thread
+// per 24 KB weight tile would pace the K loop.
 template <int MODE>
 __device__ __forceinline__ void mx_producer_b(const CUtensorMap* tm0, const CUtensorMap* tm1, const MxParams& p,
                                               const int* seg, const int* ipre, int total, uint32_t sbase,
-                                              uint32_t bars, volatile int* abort)
+                                              uint32_t bars, volatile int* abort, int part)
 {
     int it = 0;
     bool ok = true;
@@ -193,14 +200,12 @@ __device__ __forceinline__ void mx_producer_b(const CUtensorMap* tm0, const CUte
                 break;
             }
             const uint32_t fb = bars + 8 * (MB_FULL + s);
-            mbar_arrive_expect_tx(fb, MX_B_TILE);
-            const uint32_t dst = sbase + s * MX_STAGE + MX_A_TILE;
-            if (MODE == 0) {  // 96 gate rows, then 96 up rows, of n-tile nt
-                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * MX_HALF, w.e, fb);
-                tma_load_3d(dst + MX_B_TILE / 2, tm1, kb * MX_BK, w.nt * MX_HALF, w.e, fb);
-            } else {
-                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * MX_BN, w.e, fb);
-            }
+            mbar_arrive_expect_tx(fb, MX_B_TILE / 2);
+            const uint32_t dst = sbase + s * MX_STAGE + MX_A_TILE + part * (MX_B_TILE / 2);
+            if (MODE == 0)  // 96 gate rows, then 96 up rows, of n-tile nt
+                tma_load_3d(dst, part ? tm1 : tm0, kb * MX_BK, w.nt * MX_HALF, w.e, fb);
+            else
+                tma_load_3d(dst, tm0, kb * MX_BK, w.nt * MX_BN + part * MX_HALF, w.e, fb);
         }
     }
     if (!ok) {  // let the copies already issued land before the CTA can exit
@@ -213,7 +218,7 @@ __device__ __forceinline__ void mx_producer_b(const CUtensorMap* tm0, const CUte
 
 __device__ __forceinline__ void mx_producer_a(const CUtensorMap* tmA, const MxParams& p, const int* seg,
                                               const int* ipre, int total, uint32_t sbase, uint32_t bars,
-                                              volatile int* abort)
+                                              volatile int* abort, int part)
 {
     int it = 0;
     bool ok = true;
@@ -227,8 +232,8 @@ __device__ __forceinline__ void mx_producer_a(const CUtensorMap* tmA, const MxPa
                 break;
             }
             const uint32_t fb = bars + 8 * (MB_FULL + s);
-            mbar_arrive_expect_tx(fb, MX_A_TILE);
-            tma_load_2d(sbase + s * MX_STAGE, tmA, kb * MX_BK, row0, fb);
+            mbar_arrive_expect_tx(fb, MX_A_TILE / 2);
+            tma_load_2d(sbase + s * MX_STAGE + part * (MX_A_TILE / 2), tmA, kb * MX_BK, row0 + part * (MX_BM / 2), fb);
         }
     }
     if (!ok) {
@@ -588,7 +593,7 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < MX_STAGES; ++s) {
-            mbar_init(bars + 8 * (MB_FULL + s), 2);   // both producers: arrive + tx
+            mbar_init(bars + 8 * (MB_FULL + s), 4);   // four producer lanes: arrive + tx
             mbar_init(bars + 8 * (MB_EMPTY + s), 1);  // MMA commit
         }
         for (int s = 0; s < SF_SLOTS; ++s) {
@@ -639,11 +644,10 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
     const int total = *bad ? 0 : ipre[E];
 
     if (warp < 4) {
-        if ((threadIdx.x & 31) == 0) {
-            if (warp == 0) mx_producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total, sbase, bars, abort);
-            else if (warp == 1) mx_mma(p, seg, ipre, total, sbase, bars, tmem, abort);
-            else if (warp == 3) mx_producer_a(&tmA, p, seg, ipre, total, sbase, bars, abort);
-        }
+        const int lane = threadIdx.x & 31;
+        if (warp == 0 && lane < 2) mx_producer_b<MODE>(&tmB0, &tmB1, p, seg, ipre, total, sbase, bars, abort, lane);
+        else if (warp == 3 && lane < 2) mx_producer_a(&tmA, p, seg, ipre, total, sbase, bars, abort, lane);
+        else if (warp == 1 && lane == 0) mx_mma(p, seg, ipre, total, sbase, bars, tmem, abort);
         if (warp == 2) mx_sf_loader<MODE>(p, seg, ipre, total, sbase + MX_OFF_SFS, bars, abort);
     } else if (warp < 8) {
         mx_epilogue<MODE>(p, seg, ipre, total, bars, tmem, abort);
@@ -817,9 +821,9 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
 
-    // 2. tensor maps: activations and intermediate [rows, K] with 128-row
-    // boxes; gate/up weights with 96-row boxes (96 gate + 96 up rows per
-    // tile), down weights with 192-row boxes.  The intermediate's map is I
+    // 2. tensor maps: activations and intermediate [rows, K] with 64-row
+    // boxes (two per tile); gate/up and down weights with 96-row boxes (96
+    // gate + 96 up rows, or two halves of 192 down rows, per tile).  The intermediate's map is I
     // wide over rows of Ip bytes, so the padding columns of the last K block
     // read as zero.
     CUtensorMap tmA1, tmG, tmU, tmA2, tmD;
@@ -832,11 +836,11 @@ cudaError_t launch_grouped_ffn_mx(const FfnMxArgs& a, cudaStream_t s)
         const uint64_t sH[1] = {static_cast<uint64_t>(Ip)};
         const uint64_t dD[3] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H), static_cast<uint64_t>(E)};
         const uint64_t sD[2] = {static_cast<uint64_t>(I), static_cast<uint64_t>(H) * I};
-        if (!a.down_only && (!make_tmap_u8(&tmA1, a.a_sorted, 2, dA, sA, 128) ||
+        if (!a.down_only && (!make_tmap_u8(&tmA1, a.a_sorted, 2, dA, sA, MX_BM / 2) ||
                              !make_tmap_u8(&tmG, a.w_gate, 3, dW, sW, MX_HALF) ||
                              !make_tmap_u8(&tmU, a.w_up, 3, dW, sW, MX_HALF)))
             return cudaErrorNotSupported;
-        if (!make_tmap_u8(&tmA2, a.h_codes, 2, dH, sH, 128) || !make_tmap_u8(&tmD, a.w_down, 3, dD, sD, MX_BN))
+        if (!make_tmap_u8(&tmA2, a.h_codes, 2, dH, sH, MX_BM / 2) || !make_tmap_u8(&tmD, a.w_down, 3, dD, sD, MX_HALF))
             return cudaErrorNotSupported;
     }
     const int grid = di.sm_count;
