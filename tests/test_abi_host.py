@@ -82,6 +82,62 @@ def test_ffn_validation(L):
     assert _ffn(L) == 5                 # no device here
 
 
+def test_quant_mx_validation(L):
+    assert L.moe_quant_act_mx(A, 4, 100, A, A, None) == 1           # H % 32 != 0
+    assert L.moe_quant_act_mx(A, 4, 16, A, A, None) == 1            # H < 32
+    assert L.moe_quant_act_mx(A, -1, 64, A, A, None) == 1
+    assert L.moe_quant_act_mx(A, 4, 64, MIS, A, None) == 3
+    assert L.moe_quant_act_mx(A, 0, 64, A, A, None) == 0             # T = 0: no-op
+    assert L.moe_quant_act_mx(A, 4, 64, A, A, None) == 5             # no device here
+
+
+def _ffn_mx(L, T=4, H=256, k=2, E=8, I=128, ws=None, ptr=A):
+    if ws is None:
+        ws = L.moe_ffn_mx_workspace_bytes(T, H, I, E, k)
+    return L.moe_grouped_ffn_mx(ptr, A, T, H, A, A, k, A, A, E, I, A, A, A, A, A, A, A, A, ws, None, None)
+
+
+def test_ffn_mx_validation(L):
+    assert _ffn_mx(L, H=200) == 1       # H % 128 != 0
+    assert _ffn_mx(L, I=96) == 1        # I < 128
+    assert _ffn_mx(L, I=144) == 2       # I % 32 != 0: unsupported (one scale per 32 columns)
+    assert _ffn_mx(L, I=16384) == 1
+    assert _ffn_mx(L, k=0) == 1
+    assert _ffn_mx(L, k=9, E=8) == 1
+    assert _ffn_mx(L, ptr=MIS) == 3
+    assert _ffn_mx(L, ws=64) == 4
+    assert _ffn_mx(L) == 5              # no device here
+    ws = L.moe_combine_workspace_bytes()
+    assert L.moe_debug_grouped_down_mx(A, A, 4, 256, 2, A, A, A, 8, 144, A, A, A, A, ws, None) == 2
+    assert L.moe_debug_grouped_down_mx(A, A, 4, 256, 2, A, A, A, 8, 128, A, A, A, A, 8, None) == 4
+
+
+def test_pack_scales_validation(L):
+    assert L.moe_mx_packed_scales_bytes(3, 70, 5120) == 3 * 10 * 70 * 16
+    assert L.moe_mx_packed_scales_bytes(2, 33, 192) == 2 * 1 * 33 * 16
+    assert L.moe_mx_packed_scales_bytes(1, 5, 100) == 0             # K % 32 != 0
+    assert L.moe_mx_pack_scales(A, 2, 33, 100, A, None) == 1
+    assert L.moe_mx_pack_scales(A, 2, 0, 192, A, None) == 1
+    assert L.moe_mx_pack_scales(A, 2, 33, 192, MIS, None) == 3
+    assert L.moe_mx_pack_scales(A, 0, 33, 192, A, None) == 0         # E = 0: no-op
+    assert L.moe_mx_pack_scales(A, 2, 33, 192, A, None) == 5         # no device here
+
+
+def test_mx_workspace_layout(L):
+    """The MX FFN workspace holds the expert-ordered codes, the intermediate
+    and both K-group-major scale arrays; the intermediate accessor points
+    inside it, at offsets that grow with T."""
+    T, H, I, E, k = 4096, 5120, 1536, 256, 8
+    P = T * k
+    b = L.moe_ffn_mx_workspace_bytes(T, H, I, E, k)
+    Ip = 1536
+    assert b >= P * (H + Ip) + P * 16 * ((H + 511) // 512 + (Ip + 511) // 512)
+    hc, hs = V(), V()
+    assert L.moe_ffn_mx_intermediate(A, T, H, I, k, ctypes.byref(hc), ctypes.byref(hs)) == 0
+    assert A.value < hc.value < hs.value < A.value + b
+    assert hs.value - hc.value >= P * Ip
+
+
 def test_combine_validation(L):
     ws = L.moe_combine_workspace_bytes()
     f = ctypes.c_float(1.0)
