@@ -77,14 +77,16 @@ constexpr int MB_FULL = 0;                       // [stages]: both producers (ar
 constexpr int MB_EMPTY = MB_FULL + MX_STAGES;    // [stages]: MMA commit
 constexpr int MB_SFF = MB_EMPTY + MX_STAGES;     // [slots]: the four stager warps
 constexpr int MB_SFE = MB_SFF + SF_SLOTS;        // [slots]: MMA commit
-constexpr int MB_SSF = MB_SFE + SF_SLOTS;        // [slots]: scale loader filled the shared slot
-constexpr int MB_SSE = MB_SSF + SF_SLOTS;        // [slots]: the four writers read it
-constexpr int MB_AF = MB_SSE + SF_SLOTS;         // [2]: accumulator full (MMA commit)
+constexpr int SG_SLOTS = 3;                      // shared ring of scale groups (four K blocks each)
+constexpr int MB_SSF = MB_SFE + SF_SLOTS;        // [SG_SLOTS]: the loader's 32 lanes' copies landed
+constexpr int MB_SSE = MB_SSF + SG_SLOTS;        // [SG_SLOTS]: the four writers read the group
+constexpr int MB_AF = MB_SSE + SG_SLOTS;         // [2]: accumulator full (MMA commit)
 constexpr int MB_AE = MB_AF + 2;                 // [2]: accumulator drained (four epilogue warps)
 constexpr int MB_N = MB_AE + 2;
 constexpr int SF_WORDS = 10;                   // per lane and K block: 4 A + 6 B scale words
-constexpr int MX_OFF_SFS = MX_STAGES * MX_STAGE;  // shared scale ring [slot][word][lane]
-constexpr int MX_OFF_BARS = MX_OFF_SFS + SF_SLOTS * SF_WORDS * 32 * 4;
+constexpr int SG_BYTES = SF_WORDS * 32 * 16;   // one group: [word][lane][4 K blocks] 32-bit words
+constexpr int MX_OFF_SFS = MX_STAGES * MX_STAGE;  // shared ring of scale groups
+constexpr int MX_OFF_BARS = MX_OFF_SFS + SG_SLOTS * SG_BYTES;
 constexpr int MX_OFF_MISC = MX_OFF_BARS + MB_N * 8;
 constexpr int MX_OFF_SEG = MX_OFF_MISC + 16;  // [E+1] offsets, then [E+1] item prefix
 constexpr int mx_smem_bytes(int E) { return MX_OFF_SEG + 2 * (E + 1) * 4 + 1024; }
@@ -249,7 +251,7 @@ __device__ __forceinline__ void mx_producer_a(const CUtensorMap* tmA, const MxPa
 // four K chunks (one K block) per 32-bit word.  Both operands' scales are
 // K-group-major ([groups][rows][16 bytes], a group = four K blocks), so the
 // loader fetches a group of four K blocks of 32 consecutive rows with one
-// coalesced 16-byte-per-lane load.  A cursor walks this CTA's (item, group)
+// coalesced 16-byte-per-lane copy.  A cursor walks this CTA's (item, group)
 // sequence.
 struct SfGroup {
     int item, kb0, row0;
@@ -269,151 +271,132 @@ __device__ __forceinline__ void sf_group_next(SfGroup& c, const MxParams& p, con
     }
 }
 
-// Chunks at or beyond nvalid of the 16-byte group starting at chunk c0 read
-// as 127 (2^0): K padding, whose codes are zero.
-__device__ __forceinline__ uint4 mask_sf16(uint4 v, int c0, int nvalid)
+// Chunks at or beyond nvalid of the 32-bit word of K block kb (chunks 4kb ..
+// 4kb+3) read as 127 (2^0): K padding, whose codes are zero.
+__device__ __forceinline__ uint32_t mask_sf4(uint32_t w, int kb, int nvalid)
 {
-    if (c0 + 16 <= nvalid) return v;
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const int c0 = 4 * kb;
+    if (c0 + 4 <= nvalid) return w;
 #pragma unroll
-    for (int b = 0; b < 16; ++b)
-        if (c0 + b >= nvalid) w[b >> 2] = (w[b >> 2] & ~(0xFFu << (8 * (b & 3)))) | (0x7Fu << (8 * (b & 3)));
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    for (int b = 0; b < 4; ++b)
+        if (c0 + b >= nvalid) w = (w & ~(0xFFu << (8 * b))) | (0x7Fu << (8 * b));
+    return w;
 }
 
-template <int MODE>
-__device__ __forceinline__ void sf_load_group(uint4 (&v)[SF_WORDS], const SfGroup& c, const MxParams& p, int total,
-                                              int lane)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes)
 {
-    if (c.item >= total) return;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        int64_t m = c.row0 + lane + 32 * j;
-        m = m < p.P ? m : p.P - 1;
-        // one 128-byte line per 8 lanes: the A scales are K-group-major
-        v[j] = mask_sf16(__ldg(reinterpret_cast<const uint4*>(p.a_sf + ((c.kb0 >> 2) * p.P + m) * 16)), 4 * c.kb0,
-                         p.a_chunks);
-    }
-#pragma unroll
-    for (int j = 0; j < 6; ++j) {
-        const uint8_t* base;
-        int row;
-        if (MODE == 0) {  // B rows 0..95 gate, 96..191 up
-            base = j < 3 ? p.b_sf0 : p.b_sf1;
-            row = c.w.nt * MX_HALF + lane + 32 * (j % 3);
-        } else {
-            base = p.b_sf0;
-            row = c.w.nt * MX_BN + lane + 32 * j;
-        }
-        const int64_t gw = (static_cast<int64_t>(c.w.e) * p.num_groups + (c.kb0 >> 2)) * p.b_rows + row;
-        v[4 + j] = row < p.b_rows ? mask_sf16(__ldg(reinterpret_cast<const uint4*>(base + gw * 16)), 4 * c.kb0,
-                                              p.b_chunks)
-                                  : make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);  // padding rows
-    }
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
-// Scale loader (warp 2, all lanes): writes each K block's words into the
-// shared slot it % SF_SLOTS, laid out [word][lane] (conflict-free), with the
-// next group's loads already in flight.  It issues no tcgen05 operation: a
-// tcgen05 wait also waits for the warp's outstanding global loads, so the
-// warps that write TMEM keep none.
-__device__ __forceinline__ bool sf_put(const uint4 (&v)[SF_WORDS], int i, int it, uint32_t sfs, uint32_t bars,
-                                       volatile int* abort)
-{
-    const int ss = it % SF_SLOTS;
-    if (!__all_sync(0xFFFFFFFFu,
-                    mbar_wait_bounded(bars + 8 * (MB_SSE + ss), ((it / SF_SLOTS) & 1) ^ 1, abort, MX_WAIT_NS)))
-        return false;
-    const int lane = threadIdx.x & 31;
-    const uint32_t slot = sfs + ss * (SF_WORDS * 32 * 4) + lane * 4;
-#pragma unroll
-    for (int j = 0; j < SF_WORDS; ++j) {
-        const uint32_t w = i == 0 ? v[j].x : i == 1 ? v[j].y : i == 2 ? v[j].z : v[j].w;
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(slot + j * 128), "r"(w) : "memory");
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bars + 8 * (MB_SSF + ss));
-    return true;
-}
-
-// Put the K blocks of one group (at most four; fewer at an item's end).
-__device__ __forceinline__ bool sf_put_group(const uint4 (&v)[SF_WORDS], int nk, int& it, uint32_t sfs,
-                                             uint32_t bars, volatile int* abort)
-{
-    for (int i = 0; i < nk; ++i, ++it)
-        if (!sf_put(v, i, it, sfs, bars, abort)) return false;
-    return true;
-}
-
+// Scale loader (warp 2, all lanes): per group of four K blocks, lane t
+// copies the 16-byte group words of A rows t + 32j (j < 4) and B rows
+// t + 32j (j < 6) straight into shared slot g % SG_SLOTS with cp.async, laid
+// out [word][lane][16 B], and the copies' completion arrives on the slot's
+// barrier (no registers in between, so three groups are in flight).  Rows
+// past the weights are zero-filled (a finite scale for zero codes).  The
+// loader issues no tcgen05 operation: a tcgen05 wait also waits for the
+// warp's outstanding global loads, so the warps that write TMEM keep none.
 template <int MODE>
 __device__ __forceinline__ void mx_sf_loader(const MxParams& p, const int* seg, const int* ipre, int total,
                                              uint32_t sfs, uint32_t bars, volatile int* abort)
 {
     const int lane = threadIdx.x & 31;
-    const int n_items = static_cast<int>(blockIdx.x) < total ? (total - 1 - static_cast<int>(blockIdx.x)) /
-                                                                      static_cast<int>(gridDim.x) + 1
-                                                                : 0;
-    const int steps = n_items * p.num_kb;
-    if (steps == 0) return;
+    if (static_cast<int>(blockIdx.x) >= total) return;
     SfGroup c;
     c.item = blockIdx.x;
     c.kb0 = 0;
     c.w = mx_decode(seg, ipre, p.E, c.item);
     c.row0 = seg[c.w.e] + c.w.mt * MX_BM;
-    uint4 g0[SF_WORDS], g1[SF_WORDS];
-    int n0 = min(4, p.num_kb - c.kb0);
-    sf_load_group<MODE>(g0, c, p, total, lane);
-    sf_group_next(c, p, seg, ipre, total);
-    int n1 = min(4, p.num_kb - c.kb0);
-    sf_load_group<MODE>(g1, c, p, total, lane);
-    sf_group_next(c, p, seg, ipre, total);
-    int it = 0;
-    while (it < steps) {
-        // put group 0, refill it with the group after next; then group 1
-        if (!sf_put_group(g0, n0, it, sfs, bars, abort)) return;
-        n0 = min(4, p.num_kb - c.kb0);
-        sf_load_group<MODE>(g0, c, p, total, lane);
-        sf_group_next(c, p, seg, ipre, total);
-        if (it >= steps) break;
-        if (!sf_put_group(g1, n1, it, sfs, bars, abort)) return;
-        n1 = min(4, p.num_kb - c.kb0);
-        sf_load_group<MODE>(g1, c, p, total, lane);
+    for (int g = 0; c.item < total; ++g) {
+        const int slot = g % SG_SLOTS;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SSE + slot), ((g / SG_SLOTS) & 1) ^ 1, abort,
+                                                        MX_WAIT_NS)))
+            break;
+        const uint32_t dst = sfs + slot * SG_BYTES + lane * 16;
+        const int grp = c.kb0 >> 2;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int64_t m = c.row0 + lane + 32 * j;
+            m = m < p.P ? m : p.P - 1;
+            cp_async16(dst + j * 512, p.a_sf + (static_cast<int64_t>(grp) * p.P + m) * 16, 16);
+        }
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+            const uint8_t* base;
+            int row;
+            if (MODE == 0) {  // B rows 0..95 gate, 96..191 up
+                base = j < 3 ? p.b_sf0 : p.b_sf1;
+                row = c.w.nt * MX_HALF + lane + 32 * (j % 3);
+            } else {
+                base = p.b_sf0;
+                row = c.w.nt * MX_BN + lane + 32 * j;
+            }
+            const bool in = row < p.b_rows;
+            const int64_t gw = (static_cast<int64_t>(c.w.e) * p.num_groups + grp) * p.b_rows + (in ? row : 0);
+            cp_async16(dst + (4 + j) * 512, base + gw * 16, in ? 16u : 0u);
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bars + 8 * (MB_SSF + slot))
+                     : "memory");
         sf_group_next(c, p, seg, ipre, total);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Scale writers (warps 8..11, all lanes): per K block, copy the shared slot
-// into TMEM lane 32q + t of the TMEM slot (columns 0..3 A rows t + 32j,
-// columns 8..13 B rows t + 32j) once the MMAs that read its previous
-// contents are done, then hand it to the MMA issuer.
-__device__ __forceinline__ void mx_sf_writer(int steps, uint32_t sfs, uint32_t bars, uint32_t tmem,
-                                             volatile int* abort)
+// Scale writers (warps 8..11, all lanes): per group, read this lane's words
+// of its four K blocks from the shared slot and release the slot; then per
+// K block, once the MMAs that read the TMEM slot's previous contents are
+// done, write TMEM lane 32q + t of TMEM slot it % SF_SLOTS (columns 0..3 A
+// rows t + 32j, columns 8..13 B rows t + 32j) and hand it to the issuer.
+__device__ __forceinline__ void mx_sf_writer(const MxParams& p, int n_items, uint32_t sfs, uint32_t bars,
+                                             uint32_t tmem, volatile int* abort)
 {
     const int lane = threadIdx.x & 31;
     const int q = (threadIdx.x >> 5) & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    for (int it = 0; it < steps; ++it) {
-        const int ss = it % SF_SLOTS;
-        const uint32_t ph = (it / SF_SLOTS) & 1;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SSF + ss), ph, abort, MX_WAIT_NS))) return;
-        uint32_t v[SF_WORDS];
-        const uint32_t slot = sfs + ss * (SF_WORDS * 32 * 4) + lane * 4;
+    int it = 0, g = 0;
+    for (int item = 0; item < n_items; ++item) {
+        for (int kb0 = 0; kb0 < p.num_kb; kb0 += 4, ++g) {
+            const int slot = g % SG_SLOTS;
+            if (!__all_sync(0xFFFFFFFFu,
+                            mbar_wait_bounded(bars + 8 * (MB_SSF + slot), (g / SG_SLOTS) & 1, abort, MX_WAIT_NS)))
+                return;
+            const int nk = p.num_kb - kb0 < 4 ? p.num_kb - kb0 : 4;
+            uint32_t v[SF_WORDS][4];
+            const uint32_t src = sfs + slot * SG_BYTES + lane * 16;
 #pragma unroll
-        for (int j = 0; j < SF_WORDS; ++j) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[j]) : "r"(slot + j * 128) : "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (MB_SSE + ss));
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SFE + ss), ph ^ 1, abort, MX_WAIT_NS)))
-            return;
-        tc_fence_after();
-        const uint32_t a[8] = {v[0], v[1], v[2], v[3], 0u, 0u, 0u, 0u};
-        const uint32_t b[8] = {v[4], v[5], v[6], v[7], v[8], v[9], 0u, 0u};
-        const uint32_t col = lane_base + SF_COL + ss * SF_SLOT_COLS;
-        tmem_st32x8(col, a);
-        tmem_st32x8(col + 8, b);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (MB_SFF + ss));
+            for (int j = 0; j < SF_WORDS; ++j)
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v[j][0]), "=r"(v[j][1]), "=r"(v[j][2]), "=r"(v[j][3])
+                             : "r"(src + j * 512)
+                             : "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + 8 * (MB_SSE + slot));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i >= nk) break;
+                const int kb = kb0 + i;
+                const int ss = it % SF_SLOTS;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(bars + 8 * (MB_SFE + ss), ((it / SF_SLOTS) & 1) ^ 1,
+                                                                abort, MX_WAIT_NS)))
+                    return;
+                tc_fence_after();
+                uint32_t a[8], b[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) a[j] = mask_sf4(v[j][i], kb, p.a_chunks);
+                a[4] = a[5] = a[6] = a[7] = 0u;
+#pragma unroll
+                for (int j = 0; j < 6; ++j) b[j] = mask_sf4(v[4 + j][i], kb, p.b_chunks);
+                b[6] = b[7] = 0u;
+                const uint32_t col = lane_base + SF_COL + ss * SF_SLOT_COLS;
+                tmem_st32x8(col, a);
+                tmem_st32x8(col + 8, b);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 8 * (MB_SFF + ss));
+                ++it;
+            }
+        }
     }
 }
 
@@ -599,7 +582,9 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
         for (int s = 0; s < SF_SLOTS; ++s) {
             mbar_init(bars + 8 * (MB_SFF + s), 4);    // four writer warps
             mbar_init(bars + 8 * (MB_SFE + s), 1);    // MMA commit
-            mbar_init(bars + 8 * (MB_SSF + s), 1);    // the loader warp
+        }
+        for (int s = 0; s < SG_SLOTS; ++s) {
+            mbar_init(bars + 8 * (MB_SSF + s), 32);   // the loader's 32 lanes (cp.async completion)
             mbar_init(bars + 8 * (MB_SSE + s), 4);    // four writer warps
         }
         for (int b = 0; b < 2; ++b) {
@@ -655,7 +640,7 @@ __global__ void __launch_bounds__(MX_THREADS, 1)
         const int n_items = static_cast<int>(blockIdx.x) < total
                                 ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                                 : 0;
-        mx_sf_writer(n_items * p.num_kb, sbase + MX_OFF_SFS, bars, tmem, abort);
+        mx_sf_writer(p, n_items, sbase + MX_OFF_SFS, bars, tmem, abort);
     }
 
     tc_fence_before();
